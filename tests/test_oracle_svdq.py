@@ -1,0 +1,192 @@
+"""Pins for oracle/svdq.py and oracle/prep.py against closed forms,
+brute force, special cases and the pages' qualitative claim."""
+import numpy as np
+import pytest
+
+import workloads
+from oracle import codecs, prep, svdq
+
+
+def _rng(s=0):
+    return np.random.default_rng(s)
+
+
+# ------------------------------------------------------- quantization ----
+def test_block_round_trip_of_representable_values():
+    # x = e2m1 value · 2^e with one group exponent; gs a power of two:
+    # the group amax is 6·2^e, so t = 2^e·gs/ (6/6) is exactly representable
+    rng = _rng(1)
+    M, K = 8, 64
+    codes = rng.integers(0, 16, (M, K)).astype(np.uint8)
+    codes[:, ::16] = 7                     # every group holds ±6 → amax = 6·2^e
+    e = rng.integers(-3, 4, (M, K // 16))
+    x = codecs.e2m1_decode(codes) * np.repeat(2.0 ** e, 16, axis=1)
+    gs = np.float32(4.0)
+    got_codes, got_sf = svdq.nvfp4_quantize(x.astype(np.float32), gs)
+    assert np.array_equal(got_codes & 0x7, codes & 0x7)
+    assert np.array_equal(codecs.e4m3_decode(got_sf), 2.0 ** e * 4.0)
+    assert np.array_equal(svdq.nvfp4_dequantize(got_codes, got_sf, gs), x)
+
+
+def test_quantization_error_within_format_bound():
+    rng = _rng(2)
+    x = workloads.to_bf16(rng.standard_normal((64, 256)).astype(np.float32) * 3)
+    q = svdq.quantize_act(x, None)
+    deq = svdq.nvfp4_dequantize(q["codes"], q["sf"], q["gs"])
+    d = codecs.e4m3_decode(q["sf"])
+    step = np.repeat(d / np.float64(q["gs"]), 16, axis=1)   # one E2M1 unit, in x units
+    v = np.abs(x.astype(np.float64)) / step                 # magnitude in E2M1 units
+    half_gap = np.where(v < 2, 0.25, np.where(v < 4, 0.5, 1.0))
+    bound = half_gap * step + np.maximum(v - 6, 0) * step + 1e-6 * step
+    assert np.all(np.abs(deq - x) <= bound)
+
+
+def test_tensor_scale_puts_the_amax_group_at_448():
+    x = workloads.to_bf16(_rng(3).standard_normal((32, 128)).astype(np.float32))
+    q = svdq.quantize_act(x, None)
+    assert q["gs"] == np.float32(2688) / np.float32(np.abs(x).max())
+    assert (q["sf"] == 0x7E).sum() >= 1
+    assert codecs.e4m3_decode(q["sf"]).max() == 448.0
+
+
+def test_zero_groups_give_zero_scale_and_signed_zero_codes():
+    x = np.zeros((2, 32), np.float32)
+    x[0, :16] = -0.0
+    x[1, 16:] = 1.0
+    q = svdq.quantize_act(x, None)
+    assert q["sf"][0].tolist() == [0, 0] and q["sf"][1, 0] == 0
+    assert np.all(q["codes"][0, :16] == 8) and np.all(q["codes"][0, 16:] == 0)
+    assert np.all(q["codes"][1, 16:] == 7)   # 1.0 · 2688 / 448 → 6
+    assert svdq.tensor_scale(0.0) == 1.0
+
+
+def test_all_zero_tensor_scale_is_one():
+    q = svdq.quantize_act(np.zeros((4, 16), np.float32), None)
+    assert q["gs"] == 1.0 and not q["sf"].any() and not q["codes"].any()
+
+
+def test_unit_smoothing_equals_no_smoothing_and_smoothing_divides():
+    x = workloads.to_bf16(_rng(4).standard_normal((16, 64)).astype(np.float32))
+    a = svdq.quantize_act(x, None, np.float32(100))
+    b = svdq.quantize_act(x, np.ones(64, np.float32), np.float32(100))
+    assert np.array_equal(a["codes"], b["codes"]) and np.array_equal(a["sf"], b["sf"])
+    s = np.full(64, 2.0, np.float32)              # power of two: exact halving
+    c = svdq.quantize_act(x, s, np.float32(100))
+    assert np.array_equal(c["xh"], x / 2)
+
+
+# --------------------------------------------------------- contractions ----
+def _brute_y(ca, sfa, gsa, xl, cw, sfw, gsw, L2t, bias):
+    M, K = ca.shape
+    N = cw.shape[0]
+    y = np.zeros((M, N))
+    for m in range(M):
+        for n in range(N):
+            acc = 0.0
+            for k in range(K):
+                a = codecs.e2m1_decode(ca[m, k]) * codecs.e4m3_decode(sfa[m, k // 16]) / float(gsa)
+                w = codecs.e2m1_decode(cw[n, k]) * codecs.e4m3_decode(sfw[n, k // 16]) / float(gsw)
+                acc += a * w
+            for j in range(xl.shape[1]):
+                acc += float(xl[m, j]) * float(L2t[n, j])
+            y[m, n] = acc + float(bias[n])
+    return y
+
+
+def test_svdq_linear_equals_triple_loop_on_tiny_shapes():
+    rng = _rng(6)
+    M, K, N, r = 3, 32, 5, 2
+    ca = rng.integers(0, 16, (M, K)).astype(np.uint8)
+    cw = rng.integers(0, 16, (N, K)).astype(np.uint8)
+    sfa = rng.integers(0, 0x7F, (M, K // 16)).astype(np.uint8)
+    sfw = rng.integers(0, 0x7F, (N, K // 16)).astype(np.uint8)
+    xl = rng.standard_normal((M, r))
+    L2t = rng.standard_normal((N, r))
+    bias = rng.standard_normal(N)
+    ref = _brute_y(ca, sfa, 3.0, xl, cw, sfw, 5.0, L2t, bias)
+    got = svdq.svdq_linear(ca, sfa, np.float32(3), xl, cw, sfw, np.float32(5), L2t, bias)
+    np.testing.assert_allclose(got, ref, rtol=1e-12, atol=1e-12)
+
+
+def test_lora_down_equals_loop_over_k():
+    rng = _rng(7)
+    x = workloads.to_bf16(rng.standard_normal((3, 48)).astype(np.float32))
+    s = (rng.uniform(0.5, 3.0, 48)).astype(np.float32)
+    L1t = workloads.to_bf16(rng.standard_normal((4, 48)).astype(np.float32))
+    got = svdq.lora_down(x, s, L1t)
+    for m in range(3):
+        for j in range(4):
+            acc = 0.0
+            for k in range(48):
+                xh = np.float32(np.float32(x[m, k]) * np.float32(np.float32(1) / s[k]))
+                acc += float(codecs.bf16_round(np.array([xh]))[0]) * float(L1t[j, k])
+            assert got[m, j] == pytest.approx(acc, rel=1e-12, abs=1e-12)
+
+
+def test_zero_residual_leaves_only_the_low_rank_branch():
+    # W = rank-2 matrix exactly representable by the bf16 factors → R = 0
+    rng = _rng(8)
+    K, N, r, M = 64, 32, 2, 16
+    L1t = workloads.to_bf16(rng.standard_normal((r, K)).astype(np.float32))
+    L2t = workloads.to_bf16(rng.standard_normal((N, r)).astype(np.float32))
+    bias = workloads.to_bf16(rng.standard_normal(N).astype(np.float32) * 0.01)
+    R = np.zeros((N, K), np.float32)
+    gs_w = svdq.tensor_scale(0.0)
+    cw, sfw = svdq.nvfp4_quantize(R, gs_w)
+    x = workloads.to_bf16(rng.standard_normal((M, K)).astype(np.float32))
+    q = svdq.quantize_act(x, None)
+    xl = svdq.lora_down(x, None, L1t)
+    y = svdq.svdq_linear(q["codes"], q["sf"], q["gs"], xl, cw, sfw, gs_w, L2t, bias)
+    expect = codecs.bf16_round(x).astype(np.float64) @ L1t.T.astype(np.float64) @ L2t.T.astype(np.float64) + bias
+    np.testing.assert_allclose(y, expect, rtol=1e-12, atol=1e-12)
+    assert gs_w == 1.0 and not sfw.any()
+
+
+def test_rank_zero_is_plain_nvfp4_gemm():
+    case = workloads.small_case(64, 128, 48, 0, seed=9)
+    d = workloads.draw_svdq(case)
+    layer = prep.prepare_svdq_layer(d["x_cal"], d["W"], d["bias"], 0)
+    out = svdq.svdq_forward(d["x"], layer)
+    A = svdq.nvfp4_dequantize(out["codes"], out["sf"], out["gs"])
+    W = svdq.nvfp4_dequantize(layer["codes_w"], layer["sf_w"], layer["gs_w"])
+    np.testing.assert_allclose(out["y"], A @ W.T + d["bias"], rtol=1e-12, atol=1e-12)
+    # and with no low-rank branch the residual is the whole smoothed weight
+    np.testing.assert_allclose(layer["R"], d["W"].astype(np.float64) * layer["s"].astype(np.float64)[None, :], rtol=1e-12)
+
+
+def test_prepared_layer_reconstructs_the_weight():
+    case = workloads.small_case(64, 128, 64, 16, seed=10)
+    d = workloads.draw_svdq(case)
+    L = prep.prepare_svdq_layer(d["x_cal"], d["W"], d["bias"], 16)
+    recon = (L["L2t"].astype(np.float64) @ L["L1t"].astype(np.float64) + L["R"]) / L["s"][None, :]
+    np.testing.assert_allclose(recon, d["W"], rtol=1e-10, atol=1e-12)
+    # the low-rank factors are the leading singular directions of Ŵ
+    What = d["W"] * L["s"][None, :]
+    sv = np.linalg.svd(What, compute_uv=False)
+    assert np.linalg.norm(L["R"]) == pytest.approx(np.sqrt((sv[16:] ** 2).sum()), rel=2e-2)
+
+
+def test_smoothing_factor_definition():
+    x = np.array([[1.0, -8.0], [2.0, 0.5]], np.float32)
+    W = np.array([[0.5, 0.02], [-0.25, 0.01]], np.float32)
+    s = prep.smoothing_factors(x, W)
+    np.testing.assert_allclose(s, [np.sqrt(2 / 0.5), np.sqrt(8 / 0.02)], rtol=1e-6)
+
+
+@pytest.mark.parametrize("frac,mult", [(0.01, 20.0), (0.02, 30.0)])
+def test_svd_branch_lowers_error_on_outlier_inputs(frac, mult):
+    # the pages' central claim: plain W4A4 is hurt by outliers; SVDQuant's
+    # low-rank branch absorbs them and lowers the error of the 4-bit layer
+    case = workloads.SvdqCase("outlier", 256, 1024, 256, 32, frac, mult, seed=11)
+    d = workloads.draw_svdq(case)
+    exact = d["x"].astype(np.float64) @ d["W"].T.astype(np.float64) + d["bias"]
+    err = {}
+    for r in (0, 32):
+        L = prep.prepare_svdq_layer(d["x_cal"], d["W"], d["bias"], r)
+        y = svdq.svdq_forward(d["x"], L)["y"]
+        err[r] = np.linalg.norm(y - exact) / np.linalg.norm(exact)
+    # and the un-smoothed plain W4A4 layer is the worst of all
+    L0 = prep.prepare_svdq_layer(d["x_cal"], d["W"], d["bias"], 0, smooth=False)
+    e_plain = np.linalg.norm(svdq.svdq_forward(d["x"], L0)["y"] - exact) / np.linalg.norm(exact)
+    assert err[32] < 0.8 * err[0], err
+    assert err[32] < e_plain
