@@ -34,30 +34,44 @@ def smoothing_factors(x, W, eps=1e-5):
     return np.sqrt(xmax / wmax).astype(np.float32)
 
 
-def low_rank_factors(What, r):
+def svd_of_smoothed(What):
+    """Thin SVD of Whatᵀ (K×N) = U Σ Vᵀ in fp64."""
+    return np.linalg.svd(np.asarray(What, dtype=np.float64).T, full_matrices=False)
+
+
+def low_rank_factors(What, r, svd=None):
     """Truncated SVD of What [N, K] (nn.Linear layout, y = x·Whatᵀ).
 
     Returns (L1t [r, K], L2t [N, r]) as float32 arrays holding bf16 values:
     x·Whatᵀ ≈ (x·L1)·L2 with L1 = L1tᵀ (K×r) and L2 = L2tᵀ (r×N).
+    ``svd`` may pass a precomputed ``svd_of_smoothed(What)``.
     """
     N, K = What.shape
     if r == 0:
         return np.zeros((0, K), np.float32), np.zeros((N, 0), np.float32)
     # Whatᵀ (K×N) = U Σ Vᵀ  ->  L1 = U_r √Σ (K×r), L2 = √Σ V_rᵀ (r×N)
-    U, S, Vt = np.linalg.svd(np.asarray(What, dtype=np.float64).T, full_matrices=False)
+    U, S, Vt = svd if svd is not None else svd_of_smoothed(What)
     root = np.sqrt(S[:r])
     L1 = U[:, :r] * root[None, :]
     L2 = root[:, None] * Vt[:r, :]
     return codecs.bf16_round(L1.T.astype(np.float32)), codecs.bf16_round(L2.T.astype(np.float32))
 
 
-def prepare_svdq_layer(x_cal, W, bias, r, smooth=True):
-    """Everything the W4A4 linear needs, from raw bf16 W [N, K] and x_cal."""
+def prepare_svdq_layer(x_cal, W, bias, r, smooth=True, svd_cache=None):
+    """Everything the W4A4 linear needs, from raw bf16 W [N, K] and x_cal.
+
+    ``svd_cache``: optional dict; the SVD of the smoothed weight is stored in
+    it under key "svd" and reused (for sweeping r over one weight)."""
     W = np.asarray(W, dtype=np.float64)
     N, K = W.shape
     s = smoothing_factors(x_cal, W) if smooth else None
     What = W * (s.astype(np.float64)[None, :] if s is not None else 1.0)
-    L1t, L2t = low_rank_factors(What, r)
+    svd = None
+    if svd_cache is not None and r > 0:
+        if "svd" not in svd_cache:
+            svd_cache["svd"] = svd_of_smoothed(What)
+        svd = svd_cache["svd"]
+    L1t, L2t = low_rank_factors(What, r, svd)
     R = What - L2t.astype(np.float64) @ L1t.astype(np.float64)   # N×K
     R32 = R.astype(np.float32)
     gs_w = svdq.tensor_scale(np.abs(R32).max())

@@ -1,0 +1,220 @@
+// awq.cu — awq_w4a16_linear: int4-weight (group 64, fp16 scale and zero)
+// by bf16-activation linear for M <= 8 rows, the bandwidth-bound modulation
+// layers of the pages (ainews.surl.tw paragraph 2: "more sensitive modulation
+// layers, or those limited by memory bandwidth, use AWQ W4A16").
+//
+// The kernel is bound by the weight stream (0.5 B/weight + 4 B per 64
+// weights of scale and zero).  Dequantizing in registers with fp32 FMAs
+// would cost M FMAs per weight on the CUDA cores (12+ us at M = 8 for a
+// 3072 x 18432 layer, above the ~5 us HBM time), so the contraction runs on
+// the tensor cores through mma.sync.m16n8k16 (bf16 in, fp32 accumulate), with
+// the weights as the 16-row A operand taken straight from registers and the
+// (tiny) activation as the B operand:
+//   * per lane, one 8-byte load per weight row and 64-wide group: 16 nibbles;
+//     nibble pairs (j, j+4) become bf16 pairs 128+q with one LOP3, and one
+//     bf16x2 subtract of (128+z) gives the exact integers q − z;
+//   * each group's partial product (4 MMAs, k = 64) is scaled by its fp16
+//     scale in fp32, so the integer weights stay exact;
+//   * x̂ = x·(1/a) is split into bf16 hi + lo parts (two B columns) so the
+//     activation keeps ~16 significant bits; for M <= 4 hi and lo share one
+//     8-column B tile, for 4 < M <= 8 they take two.
+// The k order inside an MMA is permuted to match the nibble pairs; the B
+// fragments are built once per CTA in shared memory in that order.
+#include "internal.h"
+#include "ptx.cuh"
+
+namespace svdq {
+namespace {
+
+constexpr int kWarps = 8;
+constexpr int kThreads = 32 * kWarps;
+constexpr int kUnroll = 4;  // groups whose loads are in flight together
+
+__device__ __forceinline__ uint32_t bf16x2_bits(float lo, float hi) {
+  __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+
+__device__ __forceinline__ uint32_t bsub2(uint32_t a, uint32_t b) {
+  __nv_bfloat162 r = __hsub2(*reinterpret_cast<__nv_bfloat162*>(&a),
+                             *reinterpret_cast<__nv_bfloat162*>(&b));
+  return *reinterpret_cast<uint32_t*>(&r);
+}
+
+__device__ __forceinline__ void mma_bf16(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                         uint32_t a3, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+template <int NT>
+__global__ void __launch_bounds__(kThreads)
+    awq_w4a16_kernel(const uint16_t* __restrict__ x, int M, int K,
+                     const float* __restrict__ ainv, const uint32_t* __restrict__ qw,
+                     const __half* __restrict__ scales, const __half* __restrict__ zeros,
+                     const uint16_t* __restrict__ bias, int N, uint16_t* __restrict__ y) {
+  extern __shared__ uint2 bfrag[];  // [K/64][4 steps][32 lanes][NT]
+  const int groups = K / 64;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int g = lane >> 2, t = lane & 3;
+
+  // ---- B fragments: column c of tile j holds token m's hi or lo part ----
+  for (int e = threadIdx.x; e < groups * 4 * 32 * NT; e += kThreads) {
+    const int j = e % NT;
+    const int ln = (e / NT) & 31;
+    const int s = (e / NT / 32) & 3;
+    const int G = e / NT / 128;
+    const int gg = ln >> 2, tt = ln & 3;
+    int m, part;
+    if (NT == 1) {
+      m = gg & 3;
+      part = gg >> 2;
+    } else {
+      m = gg;
+      part = j;
+    }
+    const int w = s >> 1, h = s & 1;
+    const int kb = 64 * G + 16 * tt + 8 * w + 2 * h;
+    const int ks[4] = {kb, kb + 4, kb + 1, kb + 5};
+    float v[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      float xv = 0.0f;
+      if (m < M) {
+        xv = __uint_as_float(static_cast<uint32_t>(x[m * K + ks[q]]) << 16);
+        if (ainv) xv = __fmul_rn(xv, ainv[ks[q]]);
+        const float hi = __bfloat162float(__float2bfloat16_rn(xv));
+        xv = part == 0 ? hi : __fsub_rn(xv, hi);
+      }
+      v[q] = xv;
+    }
+    bfrag[e] = make_uint2(bf16x2_bits(v[0], v[1]), bf16x2_bits(v[2], v[3]));
+  }
+  __syncthreads();
+
+  const int ntiles = N / 16;
+  for (int tile = blockIdx.x * kWarps + warp; tile < ntiles; tile += gridDim.x * kWarps) {
+    const int n_a = tile * 16 + g, n_b = n_a + 8;
+    const uint2* qa = reinterpret_cast<const uint2*>(qw + static_cast<size_t>(n_a) * (K / 8)) + t;
+    const uint2* qb = reinterpret_cast<const uint2*>(qw + static_cast<size_t>(n_b) * (K / 8)) + t;
+    const __half* sa = scales + static_cast<size_t>(n_a) * groups;
+    const __half* sb = scales + static_cast<size_t>(n_b) * groups;
+    const __half* za = zeros + static_cast<size_t>(n_a) * groups;
+    const __half* zb = zeros + static_cast<size_t>(n_b) * groups;
+    float acc[NT][4] = {};
+    for (int G0 = 0; G0 < groups; G0 += kUnroll) {
+      uint2 wa[kUnroll], wb[kUnroll];
+      float sca[kUnroll], scb[kUnroll], zfa[kUnroll], zfb[kUnroll];
+#pragma unroll
+      for (int u = 0; u < kUnroll; ++u) {
+        const int G = G0 + u;
+        if (G < groups) {
+          wa[u] = __ldcs(qa + G * 4);  // 4 lanes x 8 B = one 32-byte sector per row and group
+          wb[u] = __ldcs(qb + G * 4);
+          sca[u] = __half2float(sa[G]);
+          scb[u] = __half2float(sb[G]);
+          zfa[u] = __half2float(za[G]);
+          zfb[u] = __half2float(zb[G]);
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < kUnroll; ++u) {
+        const int G = G0 + u;
+        if (G >= groups) break;
+        const uint32_t za2 = bf16x2_bits(128.0f + zfa[u], 128.0f + zfa[u]);
+        const uint32_t zb2 = bf16x2_bits(128.0f + zfb[u], 128.0f + zfb[u]);
+        float cg[NT][4] = {};
+        const uint2* bf = bfrag + static_cast<size_t>(G) * 4 * 32 * NT;
+#pragma unroll
+        for (int w = 0; w < 2; ++w) {
+          const uint32_t Wa = w ? wa[u].y : wa[u].x;
+          const uint32_t Wb = w ? wb[u].y : wb[u].x;
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const int s = 2 * w + h;
+            const uint32_t a0 = bsub2(((Wa >> (8 * h)) & 0x000F000Fu) | 0x43004300u, za2);
+            const uint32_t a2 = bsub2(((Wa >> (8 * h + 4)) & 0x000F000Fu) | 0x43004300u, za2);
+            const uint32_t a1 = bsub2(((Wb >> (8 * h)) & 0x000F000Fu) | 0x43004300u, zb2);
+            const uint32_t a3 = bsub2(((Wb >> (8 * h + 4)) & 0x000F000Fu) | 0x43004300u, zb2);
+#pragma unroll
+            for (int j = 0; j < NT; ++j) {
+              const uint2 b = bf[(s * 32 + lane) * NT + j];
+              mma_bf16(cg[j], a0, a1, a2, a3, b.x, b.y);
+            }
+          }
+        }
+#pragma unroll
+        for (int j = 0; j < NT; ++j) {
+          acc[j][0] = fmaf(cg[j][0], sca[u], acc[j][0]);
+          acc[j][1] = fmaf(cg[j][1], sca[u], acc[j][1]);
+          acc[j][2] = fmaf(cg[j][2], scb[u], acc[j][2]);
+          acc[j][3] = fmaf(cg[j][3], scb[u], acc[j][3]);
+        }
+      }
+    }
+    // c0,c1: row n_a, columns 2t, 2t+1; c2,c3: row n_b, same columns
+    float r0, r1, r2, r3;
+    int m_first;
+    bool store;
+    if (NT == 1) {
+      // columns 0-3 hold the hi parts of tokens 0-3, columns 4-7 the lo parts
+      r0 = acc[0][0] + __shfl_xor_sync(0xffffffffu, acc[0][0], 2);
+      r1 = acc[0][1] + __shfl_xor_sync(0xffffffffu, acc[0][1], 2);
+      r2 = acc[0][2] + __shfl_xor_sync(0xffffffffu, acc[0][2], 2);
+      r3 = acc[0][3] + __shfl_xor_sync(0xffffffffu, acc[0][3], 2);
+      m_first = 2 * t;
+      store = t < 2;
+    } else {
+      r0 = acc[0][0] + acc[NT - 1][0];
+      r1 = acc[0][1] + acc[NT - 1][1];
+      r2 = acc[0][2] + acc[NT - 1][2];
+      r3 = acc[0][3] + acc[NT - 1][3];
+      m_first = 2 * t;
+      store = true;
+    }
+    if (store) {
+      const float ba = bias ? __uint_as_float(static_cast<uint32_t>(bias[n_a]) << 16) : 0.0f;
+      const float bb = bias ? __uint_as_float(static_cast<uint32_t>(bias[n_b]) << 16) : 0.0f;
+      const float out[2][2] = {{r0, r2}, {r1, r3}};
+#pragma unroll
+      for (int i = 0; i < 2; ++i) {
+        const int m = m_first + i;
+        if (m < M) {
+          __nv_bfloat16 va = __float2bfloat16_rn(out[i][0] + ba);
+          __nv_bfloat16 vb = __float2bfloat16_rn(out[i][1] + bb);
+          y[static_cast<size_t>(m) * N + n_a] = *reinterpret_cast<uint16_t*>(&va);
+          y[static_cast<size_t>(m) * N + n_b] = *reinterpret_cast<uint16_t*>(&vb);
+        }
+      }
+    }
+  }
+}
+
+}  // namespace
+
+svdq_status launch_awq_w4a16(const LaunchCtx& ctx, const void* x, int64_t M, int64_t K,
+                             const float* act_scale_inv, const uint32_t* qweight,
+                             const void* scales, const void* zeros, const void* bias, int64_t N,
+                             void* y) {
+  const int ntiles = static_cast<int>(N / 16);
+  const int grid = std::max(1, std::min((ntiles + kWarps - 1) / kWarps, 2 * ctx.num_sms));
+  const int nt = M <= 4 ? 1 : 2;
+  const size_t smem = static_cast<size_t>(K) * 16 * nt;
+  static bool attr_done[2][64] = {};
+  if (!attr_done[nt - 1][ctx.device & 63]) {
+    cudaFuncSetAttribute(nt == 1 ? awq_w4a16_kernel<1> : awq_w4a16_kernel<2>,
+                         cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
+    attr_done[nt - 1][ctx.device & 63] = true;
+  }
+  auto kern = nt == 1 ? awq_w4a16_kernel<1> : awq_w4a16_kernel<2>;
+  kern<<<grid, kThreads, smem, ctx.stream>>>(
+      static_cast<const uint16_t*>(x), static_cast<int>(M), static_cast<int>(K), act_scale_inv,
+      qweight, static_cast<const __half*>(scales), static_cast<const __half*>(zeros),
+      static_cast<const uint16_t*>(bias), static_cast<int>(N), static_cast<uint16_t*>(y));
+  return check_launch("awq_w4a16_kernel");
+}
+
+}  // namespace svdq

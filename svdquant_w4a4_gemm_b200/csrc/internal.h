@@ -1,0 +1,50 @@
+// internal.h — host-side plumbing shared by the library's translation units.
+#pragma once
+
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "svdq.h"
+
+namespace svdq {
+
+// Per-launch context the API layer fills in after validation.
+struct LaunchCtx {
+  cudaStream_t stream;
+  int device;
+  int num_sms;
+  uint32_t* err_word;    // device error word of `device`
+  uint64_t timeout_ns;   // bound on every in-kernel wait
+  int fault_flags;       // test-only fault injection
+};
+
+// Encode a 2-D tiled tensor map (row-major [rows, cols] of `elem_bytes`
+// elements, row stride `row_stride_bytes`), box [box_rows, box_cols].
+// swizzle_bytes: 0, 32, 64 or 128.  Returns false and sets the detail on error.
+bool make_tmap_2d(CUtensorMap* map, const void* base, CUtensorMapDataType dtype,
+                  uint32_t elem_bytes, uint64_t rows, uint64_t cols, uint64_t row_stride_bytes,
+                  uint32_t box_rows, uint32_t box_cols, int swizzle_bytes);
+
+// Thread-local error detail (api.cu).
+svdq_status fail(svdq_status st, const char* fmt, ...);
+svdq_status check_launch(const char* what);
+
+// Kernel launchers (one per translation unit).  Arguments are validated.
+svdq_status launch_quantize_act(const LaunchCtx& ctx, const void* x, int64_t M, int64_t K,
+                                int64_t ldx, const float* smooth_s, const void* L1t, int r,
+                                const float* act_gscale, float* act_gscale_out, uint8_t* q_out,
+                                uint8_t* sf_out, float* lora_out);
+
+svdq_status launch_w4a4_gemm(const LaunchCtx& ctx, const uint8_t* q_act, const uint8_t* sf_act,
+                             const float* act_gscale, const float* lora_act, const uint8_t* q_w,
+                             const uint8_t* sf_w, const float* w_gscale, const void* L2t, int r,
+                             const void* bias, int64_t M, int64_t N, int64_t K, void* y,
+                             int64_t ldy);
+
+svdq_status launch_awq_w4a16(const LaunchCtx& ctx, const void* x, int64_t M, int64_t K,
+                             const float* act_scale_inv, const uint32_t* qweight,
+                             const void* scales, const void* zeros, const void* bias, int64_t N,
+                             void* y);
+
+}  // namespace svdq

