@@ -1,0 +1,435 @@
+"""Benchmark of the SVDQuant W4A4 (NVFP4) linear on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference] [--legs]
+
+One step = one pass of the layer over one batch: the quantize call
+(smoothing + NVFP4 activation quantization + low-rank down-projection) and
+the W4A4 GEMM call (block-scaled FP4 MMA + low-rank up-projection + bias +
+bf16 store), on the attention-projection workload M=4096 tokens, K=N=3072,
+r=32.  Prints one JSON line (rank 0).  Multi-GPU runs are independent
+replicas (weak scaling: each rank runs its own batch; the layer needs no
+exchange); timing is the max over ranks of the device-timed region.
+
+The oracle (``oracle/``, CPU) is used only by the ``cpu_baseline`` leg and
+by ``--impl reference``.
+"""
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads  # noqa: E402
+
+CASE = workloads.HEADLINE
+METRIC = "SVDQ NVFP4 linear TFLOP/s & % dense-FP4 peak (M4096 K3072 N3072 r32)"
+UNIT = "TFLOP/s"
+WORKLOAD = "attn-proj SVDQ W4A4 NVFP4 linear M4096 K3072 N3072 r32 (quantize + GEMM)"
+FP4_PER_BF16 = 4.0          # nominal dense FP4 / BF16 tensor throughput ratio (9 / 2.25 PF)
+DATASHEET_FP4_TFLOPS = 9000.0
+
+
+def layer_flops(M, K, N, r):
+    return 2.0 * M * N * K + 2.0 * M * r * (K + N)
+
+
+def peaks():
+    p = {}
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+    except OSError:
+        pass
+    return p
+
+
+# ------------------------------------------------------------------ clocks --
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.idx = gpu_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        self.lines = []
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [l for l in out.splitlines() if l.strip()]
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for l in getattr(self, "lines", []):
+            f = [x.strip() for x in l.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------- device workload --
+def make_sets(nsets, dev, seed_base=0):
+    """``nsets`` independent layers (weights + activations) prepared on the
+    device by the library's own offline prep; rotating through them keeps
+    every step's operands out of L2."""
+    import svdquant_w4a4_gemm_b200 as sv
+    from svdquant_w4a4_gemm_b200 import prep as dprep
+    d = workloads.draw_svdq(CASE)
+    x0 = torch.from_numpy(d["x"]).to(dev).to(torch.bfloat16)
+    W0 = torch.from_numpy(d["W"]).to(dev).to(torch.bfloat16)
+    b0 = torch.from_numpy(d["bias"]).to(dev).to(torch.bfloat16)
+    xc = torch.from_numpy(d["x_cal"]).to(dev).to(torch.bfloat16)
+    w0 = dprep.prepare_svdq(W0, b0, xc, CASE.r)
+    gs = torch.empty(1, device=dev)
+    sv.quantize_act(x0, w0.smooth, w0.L1t, None, out=(
+        torch.empty(CASE.M, CASE.K // 2, dtype=torch.uint8, device=dev),
+        torch.empty(sv.scale_bytes(CASE.M, CASE.K), dtype=torch.uint8, device=dev),
+        torch.empty(CASE.M, CASE.r, device=dev), gs))     # static scale from the data
+    sets = []
+    for i in range(nsets):
+        # distinct copies (same values) so that no two steps share memory
+        w = sv.SvdqWeights(q_w=w0.q_w.clone(), sf_w=w0.sf_w.clone(), gs_w=w0.gs_w.clone(),
+                           L1t=w0.L1t.clone(), L2t=w0.L2t.clone(), smooth=w0.smooth.clone(),
+                           bias=w0.bias.clone())
+        M, K, N, r = CASE.M, CASE.K, CASE.N, CASE.r
+        sets.append(dict(
+            w=w, x=x0.clone(), gs=gs.clone(),
+            q=torch.empty(M, K // 2, dtype=torch.uint8, device=dev),
+            sf=torch.empty(sv.scale_bytes(M, K), dtype=torch.uint8, device=dev),
+            lora=torch.empty(M, r, device=dev), gso=torch.empty(1, device=dev),
+            y=torch.empty(M, N, dtype=torch.bfloat16, device=dev)))
+    return sets
+
+
+def set_bytes(s):
+    return sum(t.numel() * t.element_size() for t in
+               [s["x"], s["q"], s["sf"], s["lora"], s["y"], s["w"].q_w, s["w"].sf_w, s["w"].L1t, s["w"].L2t])
+
+
+def run_step(sv, s):
+    sv.quantize_act(s["x"], s["w"].smooth, s["w"].L1t, s["gs"], out=(s["q"], s["sf"], s["lora"], s["gso"]))
+    sv.w4a4_linear(s["q"], s["sf"], s["gso"], s["lora"], s["w"], y=s["y"])
+
+
+def kernel_traffic(kernel_file, kernel_name):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken
+    on the current source of the kernel (else None)."""
+    path = os.path.join(ROOT, "profiles", "dram_traffic.json")
+    try:
+        with open(path) as f:
+            tab = json.load(f)
+        src = open(os.path.join(ROOT, "svdquant_w4a4_gemm_b200", "csrc", kernel_file), "rb").read()
+        h = hashlib.sha256(src).hexdigest()[:16]
+        ent = tab.get(kernel_name)
+        if ent and ent.get("source_sha256_16") == h:
+            return ent.get("dram_bytes_per_launch")
+    except (OSError, ValueError):
+        pass
+    return None
+
+
+def bench_device(args, rank, world, dev):
+    import svdquant_w4a4_gemm_b200 as sv
+    torch.cuda.set_device(dev)
+    props = torch.cuda.get_device_properties(dev)
+    l2 = getattr(props, "L2_cache_size", 126 * 2 ** 20) or 126 * 2 ** 20
+    probe = make_sets(1, dev)
+    per = set_bytes(probe[0])
+    nsets = max(2, int(np.ceil(3 * l2 / per)))
+    sets = probe + make_sets(nsets - 1, dev)[: nsets - 1]
+    stream = torch.cuda.current_stream(dev)
+    M, K, N, r = CASE.M, CASE.K, CASE.N, CASE.r
+
+    for i in range(args.warmup):
+        run_step(sv, sets[i % nsets])
+    sv.check_device_errors()
+
+    # ---- timed region: K steps, events around each kernel ----
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(dev)
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    with ClockSampler(props_index(dev)) as clk:
+        t_start.record(stream)
+        for i in range(args.steps):
+            s = sets[i % nsets]
+            e0, e1, e2 = ev[i]
+            e0.record(stream)
+            sv.quantize_act(s["x"], s["w"].smooth, s["w"].L1t, s["gs"],
+                            out=(s["q"], s["sf"], s["lora"], s["gso"]))
+            e1.record(stream)
+            sv.w4a4_linear(s["q"], s["sf"], s["gso"], s["lora"], s["w"], y=s["y"])
+            e2.record(stream)
+        t_end.record(stream)
+        torch.cuda.synchronize(dev)
+    if world > 1:
+        torch.distributed.barrier()
+    sv.check_device_errors()
+    total_ms = t_start.elapsed_time(t_end)
+    if world > 1:
+        t = torch.tensor([total_ms], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        total_ms = float(t.item())
+    k1_us = [e[0].elapsed_time(e[1]) * 1e3 for e in ev]
+    k2_us = [e[1].elapsed_time(e[2]) * 1e3 for e in ev]
+
+    # ---- e2e: the same call with host buffers, copies inside the timed region ----
+    x_host = sets[0]["x"].cpu().pin_memory()
+    y_host = torch.empty(M, N, dtype=torch.bfloat16).pin_memory()
+    e2e_steps = max(3, min(args.steps, 20))
+    s0 = sets[0]
+    for _ in range(2):
+        s0["x"].copy_(x_host, non_blocking=True)
+        run_step(sv, s0)
+        y_host.copy_(s0["y"], non_blocking=True)
+    torch.cuda.synchronize(dev)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for i in range(e2e_steps):
+        s = sets[i % nsets]
+        s["x"].copy_(x_host, non_blocking=True)
+        run_step(sv, s)
+        y_host.copy_(s["y"], non_blocking=True)
+    b.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = a.elapsed_time(b) / e2e_steps
+
+    legs = bench_awq_legs(sv, dev, l2) if args.legs and rank == 0 else None
+    return dict(total_ms=total_ms, k1_us=k1_us, k2_us=k2_us, clocks=clk.summary(), nsets=nsets,
+                set_mb=per / 2 ** 20, e2e_ms=e2e_ms, h2d=x_host.numel() * 2, d2h=y_host.numel() * 2,
+                legs=legs)
+
+
+def props_index(dev):
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+    idx = torch.device(dev).index or 0
+    if vis:
+        ids = [v.strip() for v in vis.split(",")]
+        if idx < len(ids) and ids[idx].isdigit():
+            return int(ids[idx])
+    return idx
+
+
+def bench_awq_legs(sv, dev, l2):
+    """The AWQ W4A16 modulation layer (M = 1, 2, 8; K = 3072, N = 18432),
+    HBM-bound: GB/s of algorithmic bytes, rotating weight copies > 3x L2."""
+    from svdquant_w4a4_gemm_b200 import prep as dprep
+    out = {}
+    for Mw, case in workloads.AWQ.items():
+        d = workloads.draw_awq(case)
+        W = torch.from_numpy(d["W"]).to(dev).to(torch.bfloat16)
+        xc = torch.from_numpy(d["x_cal"]).to(dev).to(torch.bfloat16)
+        ainv, qw, sc, z = dprep.prepare_awq(W, xc)
+        wbytes = qw.numel() * 4 + sc.numel() * 2 + z.numel() * 2
+        n = max(2, int(np.ceil(3 * l2 / wbytes)))
+        copies = [(qw.clone(), sc.clone(), z.clone()) for _ in range(n)]
+        x = torch.from_numpy(d["x"]).to(dev).to(torch.bfloat16)
+        b = torch.from_numpy(d["bias"]).to(dev).to(torch.bfloat16)
+        y = torch.empty(Mw, case.N, dtype=torch.bfloat16, device=dev)
+        for i in range(5):
+            c = copies[i % n]
+            sv.awq_w4a16_linear(x, ainv, c[0], c[1], c[2], b, y=y)
+        iters = 60
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize(dev)
+        e0.record()
+        for i in range(iters):
+            c = copies[i % n]
+            sv.awq_w4a16_linear(x, ainv, c[0], c[1], c[2], b, y=y)
+        e1.record()
+        torch.cuda.synchronize(dev)
+        us = e0.elapsed_time(e1) / iters * 1e3
+        algo = wbytes + x.numel() * 2 + ainv.numel() * 4 + b.numel() * 2 + y.numel() * 2
+        out[f"awq_M{Mw}"] = {"us": round(us, 3), "GB/s": round(algo / us / 1e3, 1),
+                             "algorithmic_bytes": int(algo)}
+    return out
+
+
+# ----------------------------------------------------------------- oracle --
+def oracle_sample(rows, seed_rows=0):
+    """Prepare the oracle's layer once and return a closure that runs the
+    oracle's whole layer on ``rows`` rows of the workload."""
+    from oracle import prep as oprep, svdq as osv
+    d = workloads.draw_svdq(CASE)
+    L = oprep.prepare_svdq_layer(d["x_cal"], d["W"], d["bias"], CASE.r)
+    gs = osv.act_tensor_scale(d["x"], L["s"])
+    xs = d["x"][seed_rows:seed_rows + rows]
+
+    def run():
+        return osv.svdq_forward(xs, L, gs)["y"]
+    return run
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads") for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return len(os.sched_getaffinity(0))
+
+
+def cpu_baseline(rows=64, reps=2):
+    run = oracle_sample(rows)
+    run()  # warm
+    t0 = time.perf_counter()
+    for _ in range(reps):
+        run()
+    dt = (time.perf_counter() - t0) / reps
+    fl = layer_flops(rows, CASE.K, CASE.N, CASE.r)
+    return {"value": fl / dt / 1e12, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+            "sample": f"{rows} of {CASE.M} rows of the layer (numpy fp64 oracle: quantize, "
+                      f"down-projection, dequantized GEMM + low-rank + bias), {reps} reps, "
+                      f"{dt:.2f} s per rep"}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return
+    rows = 32
+    run = oracle_sample(rows)
+    for _ in range(args.warmup):
+        run()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        run()
+    dt = (time.perf_counter() - t0) / args.steps
+    fl = layer_flops(rows, CASE.K, CASE.N, CASE.r)
+    v = fl / dt / 1e12
+    line = {"impl": "reference", "metric": METRIC, "value": v, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": {"workload": WORKLOAD, "M": CASE.M, "K": CASE.K,
+                                            "N": CASE.N, "r": CASE.r, "parallelism": "replicas"},
+            "cpu_baseline": {"value": v, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+                             "sample": f"{rows} of {CASE.M} rows per step"},
+            "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------- main --
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--legs", action="store_true", help="also time the AWQ W4A16 modulation layer")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+
+    # the CPU baseline runs before any CUDA work (rank 0, N = 1 only)
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline()
+
+    dev = f"cuda:{local}"
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(dev)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device(dev))
+    res = bench_device(args, rank, world, dev)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+    if rank != 0:
+        return
+
+    M, K, N, r = CASE.M, CASE.K, CASE.N, CASE.r
+    fl = layer_flops(M, K, N, r)
+    ms = res["total_ms"] / args.steps
+    value = fl * world / (ms * 1e-3) / 1e12
+    pk = peaks()
+    sustained = pk.get("bf16_tflops_sustained")
+    burst = pk.get("bf16_tflops")
+    if sustained:
+        peak, peak_src = sustained * FP4_PER_BF16, "of measured (sustained bf16 x nominal fp4/bf16 = 4)"
+    else:
+        peak, peak_src = 1590.0 * FP4_PER_BF16, "of fallback (1.59 PF bf16 x 4)"
+    k2 = statistics.mean(res["k2_us"])
+    k1 = statistics.mean(res["k1_us"])
+    achieved = fl / (k2 * 1e-6) / 1e12
+    k1_bytes = M * K * 2 + K * 4 + r * K * 2 + M * K // 2 + (M * K // 16) + M * r * 4
+    hbm = pk.get("hbm_gbs", 6650.0)
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "nvfp4", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "M": M, "K": K, "N": N, "r": r, "group": 16,
+                   "parallelism": "replicas" if world > 1 else "single",
+                   "l2": f"rotating {res['nsets']} distinct input+weight sets of "
+                         f"{res['set_mb']:.0f} MB (> 3x L2), no flush"},
+        "pct_dense_fp4_peak": {"of_measured": round(value / world / peak, 4),
+                               "of_datasheet_9PF": round(value / world / DATASHEET_FP4_TFLOPS, 4)},
+        "roofline": {"bound": "tensor", "kernel": "w4a4_gemm_kernel", "achieved": round(achieved, 1),
+                     "peak": round(peak, 1), "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
+                     "peak_source": peak_src,
+                     "traffic": kernel_traffic("gemm.cu", "w4a4_gemm_kernel"),
+                     "algorithmic_flops_per_launch": fl, "avg_launch_us": round(k2, 3)},
+        "kernels": {"quantize_act_kernel": {"avg_launch_us": round(k1, 3),
+                                            "GB/s": round(k1_bytes / k1 / 1e3, 1),
+                                            "frac_hbm": round(k1_bytes / k1 / 1e3 / hbm, 4),
+                                            "algorithmic_bytes": k1_bytes,
+                                            "traffic": kernel_traffic("quantize.cu", "quantize_act_kernel")},
+                    "w4a4_gemm_kernel": {"avg_launch_us": round(k2, 3)}},
+        "clocks": res["clocks"],
+        "e2e": {"value": fl / (res["e2e_ms"] * 1e-3) / 1e12, "unit": UNIT,
+                "h2d_bytes_per_step": res["h2d"] + 4 * 0, "d2h_bytes_per_step": res["d2h"]},
+        "gpu_launches": 2 * args.steps,
+        "cpu_baseline": cpu,
+    }
+    if res["legs"]:
+        line["legs"] = res["legs"]
+    print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

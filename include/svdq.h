@@ -116,8 +116,9 @@ svdq_status svdq_quantize_act(const void* x_bf16, int64_t M, int64_t K, int64_t 
  *   y = bf16( dec(A)·dec(W)ᵀ + lora_act·L2 + bias )
  *
  * computed as acc = Σ e2m1_a·sfa·e2m1_w·sfw (tcgen05 block-scaled FP4 MMA,
- * fp32 in TMEM) + bf16(lora_act·gs_a·gs_w)·L2 (bf16 MMA into the same
- * accumulator), y = bf16(acc/(gs_a·gs_w) + bias).
+ * fp32 in TMEM) + (hi + lo)·L2 (bf16 MMAs into the same accumulator, where
+ * hi = bf16(lora_act·gs_a·gs_w) and lo = bf16(lora_act·gs_a·gs_w − hi)),
+ * y = bf16(acc/(gs_a·gs_w) + bias).
  *
  *   q_act, sf_act, act_gscale   activation operand exactly as
  *               svdq_quantize_act writes it ([M, K/2] codes, scale buffer,
@@ -147,11 +148,14 @@ svdq_status svdq_w4a4_linear(const uint8_t* q_act, const uint8_t* sf_act,
  *
  *   y[m,n] = bf16( Σ_k (x[m,k]·act_scale_inv[k]) · (q[n,k] − z[n,k/g])·sc[n,k/g] + b[n] )
  *
- *   x_bf16        [M, K] bf16, contiguous.  1 <= M <= 8.
- *   K             K >= 64, K % 64 == 0.
- *   act_scale_inv [K] fp32 (1/a_k of the AWQ per-channel scale) or NULL.
- *   qweight       [N, K/8] uint32: nibble j (bits 4j..4j+3) of word w of row n
- *                 is q[n, 8w + j], an unsigned 0..15.
+ *   x_bf16        [M, K] bf16, contiguous, 16-byte aligned.  1 <= M <= 8.
+ *   K             K >= 64, K % 64 == 0; K <= 14464 for M <= 4 and K <= 7232
+ *                 for M > 4 (the per-CTA activation fragment table lives in
+ *                 shared memory: 16 or 32 bytes per k).
+ *   act_scale_inv [K] fp32 (1/a_k of the AWQ per-channel scale), 16-byte
+ *                 aligned, or NULL.
+ *   qweight       [N, K/8] uint32, 16-byte aligned: nibble j (bits 4j..4j+3)
+ *                 of word w of row n is q[n, 8w + j], an unsigned 0..15.
  *   scales_f16, zeros_f16   [N, K/group] fp16; zeros hold integers 0..15.
  *   group         must be 64.
  *   bias_bf16     [N] bf16 or NULL.

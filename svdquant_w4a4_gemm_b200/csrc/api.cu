@@ -261,12 +261,12 @@ svdq_status awq_w4a16_linear(const void* x_bf16, int64_t M, int64_t K, const flo
                 (long long)K, (long long)kmax, (long long)M);
   if (N < 16 || N % 16 != 0 || N > (1ll << 30))
     return fail(SVDQ_ERR_INVALID_ARG, "N=%lld must be a positive multiple of 16", (long long)N);
-  if (!aligned16(qweight)) return fail(SVDQ_ERR_MISALIGNED, "qweight must be 16-byte aligned");
-  if ((reinterpret_cast<uintptr_t>(x_bf16) & 1) || (reinterpret_cast<uintptr_t>(y_bf16) & 1) ||
-      (reinterpret_cast<uintptr_t>(scales_f16) & 1) || (reinterpret_cast<uintptr_t>(zeros_f16) & 1) ||
-      (bias_bf16 && (reinterpret_cast<uintptr_t>(bias_bf16) & 1)) ||
-      (act_scale_inv && (reinterpret_cast<uintptr_t>(act_scale_inv) & 3)))
-    return fail(SVDQ_ERR_MISALIGNED, "16-bit operands must be 2-byte and fp32 4-byte aligned");
+  if (!aligned16(qweight) || !aligned16(x_bf16) || (act_scale_inv && !aligned16(act_scale_inv)))
+    return fail(SVDQ_ERR_MISALIGNED, "x, act_scale_inv and qweight must be 16-byte aligned");
+  if ((reinterpret_cast<uintptr_t>(y_bf16) & 1) || (reinterpret_cast<uintptr_t>(scales_f16) & 1) ||
+      (reinterpret_cast<uintptr_t>(zeros_f16) & 1) ||
+      (bias_bf16 && (reinterpret_cast<uintptr_t>(bias_bf16) & 1)))
+    return fail(SVDQ_ERR_MISALIGNED, "y, scales, zeros and bias must be 2-byte aligned");
   LaunchCtx ctx{};
   if (svdq_status e = device_ctx(stream, &ctx)) return e;
   if (svdq_status e = launch_awq_w4a16(ctx, x_bf16, M, K, act_scale_inv, qweight, scales_f16,

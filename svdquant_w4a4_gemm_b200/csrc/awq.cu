@@ -28,7 +28,7 @@ namespace {
 
 constexpr int kWarps = 8;
 constexpr int kThreads = 32 * kWarps;
-constexpr int kUnroll = 4;  // groups whose loads are in flight together
+constexpr int kUnroll = 8;  // groups whose loads are in flight together
 
 __device__ __forceinline__ uint32_t bf16x2_bits(float lo, float hi) {
   __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
@@ -62,36 +62,49 @@ __global__ void __launch_bounds__(kThreads)
   const int g = lane >> 2, t = lane & 3;
 
   // ---- B fragments: column c of tile j holds token m's hi or lo part ----
-  for (int e = threadIdx.x; e < groups * 4 * 32 * NT; e += kThreads) {
+  // One item = (group G, lane, tile j): its 4 steps need x̂ at the 16
+  // contiguous k = 64G + 16·t .. +16 of one token, read with vector loads.
+  for (int e = threadIdx.x; e < groups * 32 * NT; e += kThreads) {
     const int j = e % NT;
     const int ln = (e / NT) & 31;
-    const int s = (e / NT / 32) & 3;
-    const int G = e / NT / 128;
+    const int G = e / NT / 32;
     const int gg = ln >> 2, tt = ln & 3;
-    int m, part;
-    if (NT == 1) {
-      m = gg & 3;
-      part = gg >> 2;
-    } else {
-      m = gg;
-      part = j;
-    }
-    const int w = s >> 1, h = s & 1;
-    const int kb = 64 * G + 16 * tt + 8 * w + 2 * h;
-    const int ks[4] = {kb, kb + 4, kb + 1, kb + 5};
-    float v[4];
+    const int m = NT == 1 ? (gg & 3) : gg;
+    const int part = NT == 1 ? (gg >> 2) : j;
+    const int k0 = 64 * G + 16 * tt;
+    float hi[16], lo[16];
+    if (m < M) {
+      const uint4* xv = reinterpret_cast<const uint4*>(x + static_cast<size_t>(m) * K + k0);
+      const uint4 u0 = xv[0], u1 = xv[1];
+      const uint32_t w[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
+      float av[16];
+      if (ainv) {
+        const float4* a4 = reinterpret_cast<const float4*>(ainv + k0);
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      float xv = 0.0f;
-      if (m < M) {
-        xv = __uint_as_float(static_cast<uint32_t>(x[m * K + ks[q]]) << 16);
-        if (ainv) xv = __fmul_rn(xv, ainv[ks[q]]);
-        const float hi = __bfloat162float(__float2bfloat16_rn(xv));
-        xv = part == 0 ? hi : __fsub_rn(xv, hi);
+        for (int q = 0; q < 4; ++q) {
+          const float4 a = a4[q];
+          av[4 * q] = a.x; av[4 * q + 1] = a.y; av[4 * q + 2] = a.z; av[4 * q + 3] = a.w;
+        }
       }
-      v[q] = xv;
+#pragma unroll
+      for (int q = 0; q < 16; ++q) {
+        float xv1 = __uint_as_float((q & 1) ? (w[q >> 1] & 0xFFFF0000u) : (w[q >> 1] << 16));
+        if (ainv) xv1 = __fmul_rn(xv1, av[q]);
+        hi[q] = __bfloat162float(__float2bfloat16_rn(xv1));
+        lo[q] = __fsub_rn(xv1, hi[q]);
+      }
+    } else {
+#pragma unroll
+      for (int q = 0; q < 16; ++q) hi[q] = lo[q] = 0.0f;
     }
-    bfrag[e] = make_uint2(bf16x2_bits(v[0], v[1]), bf16x2_bits(v[2], v[3]));
+#pragma unroll
+    for (int s = 0; s < 4; ++s) {
+      const int w = s >> 1, h = s & 1;
+      const int kb = 8 * w + 2 * h;  // offset of slot 2t within the 16
+      const float* v = part == 0 ? hi : lo;
+      bfrag[((G * 4 + s) * 32 + ln) * NT + j] =
+          make_uint2(bf16x2_bits(v[kb], v[kb + 4]), bf16x2_bits(v[kb + 1], v[kb + 5]));
+    }
   }
   __syncthreads();
 

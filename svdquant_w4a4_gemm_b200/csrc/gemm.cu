@@ -3,8 +3,12 @@
 // 4-bit compute kernel", blog.margrop.com "技术细节 §1", SVDQuant step 4).
 //
 //   y = bf16( α·acc + bias ),  α = 1/(gs_a·gs_w)
-//   acc = bf16(xl·gs_a·gs_w)·L2            (kind::f16 MMAs, first)
+//   acc = (hi + lo)·L2                      (kind::f16 MMAs, first)
 //       + Σ_k e2m1_a·sfa · e2m1_w·sfw      (kind::mxf4nvf4 block-scaled MMAs)
+//   hi = bf16(xl·gs_a·gs_w), lo = bf16(xl·gs_a·gs_w − hi)
+// The low-rank term can dominate y (it carries the outlier channels), so
+// its activation operand keeps ~16 significant bits through the hi/lo
+// split; L2 itself is bf16 by construction.
 //
 // One CTA computes a 128 x BN tile of y (BN = 256, or 128 when N is not a
 // multiple of 256), fp32 accumulator in tensor memory (TMEM).
@@ -19,11 +23,14 @@
 //              .warpx4, 4 columns per 128 rows per 64 K) and issues four
 //              block-scaled MMAs (K = 64 each); tcgen05.commit frees the stage.
 //   warps 2-5  first convert the [128 x r] fp32 down-projection rows into
-//              bf16(xl·gs_a·gs_w) in the A slot of the first ring stages
+//              the hi/lo bf16 parts in the A slot of the first ring stages
 //              (128-byte swizzle written by hand), then run the epilogue:
 //              TMEM -> registers, α·acc + bias, bf16, store.
 // The low-rank steps go through the same shared-memory ring as the FP4
-// stages (one ring slot per 64 of r), so they need no memory of their own.
+// stages, so they need no memory of their own: for r <= 32 one ring slot
+// holds hi in A columns [0, 32) and lo in [32, 64) against one L2ᵀ slice;
+// for r = 64, 128 each 64-wide slice of r takes two slots (hi, then lo),
+// both loading the same L2ᵀ slice.
 #include "internal.h"
 #include "ptx.cuh"
 
@@ -90,7 +97,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n0 = blockIdx.x * BN;
   const int m0 = blockIdx.y * kBM;
-  const int nlr = (p.r + 63) / 64;           // low-rank ring steps
+  const bool lr_packed = p.r > 0 && p.r <= 32;  // hi and lo share one A tile
+  const int nlr = p.r == 0 ? 0 : (lr_packed ? 1 : 2 * (p.r / 64));  // low-rank ring steps
   const int kblocks = p.K / 64;              // 64-element K blocks (one MMA each)
   const int nk = (kblocks + 3) / 4;          // FP4 ring steps (256 K each, last may be short)
   const int nsteps = nlr + nk;
@@ -129,9 +137,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!mbar_wait(&empty[s], ph ^ 1, p.wait, kErrTimeoutEmpty)) break;
         if (p.fault == 1 && i == 0) continue;  // test hook: this stage never fills
         if (i < nlr) {
-          // L2ᵀ[n0 .. n0+BN) x r[64i .. 64i+64) as bf16, zero-filled past r
+          // L2ᵀ[n0 .. n0+BN) x r[64c .. 64c+64) as bf16, zero-filled past r
+          const int c = lr_packed ? 0 : i / 2;
           mbar_arrive_expect_tx(&full[s], L::kB);
-          tma_load_2d(stage_b(s), &tmap_l2, &full[s], 64 * i, n0);
+          tma_load_2d(stage_b(s), &tmap_l2, &full[s], 64 * c, n0);
         } else {
           const int kb = i - nlr;  // 256-element K step
           const int nkb = min(4, kblocks - 4 * kb);                  // scale blocks (MMAs) in it
@@ -173,11 +182,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t a0 = smem_u32(stage_a(s));
         const uint32_t b0 = smem_u32(stage_b(s));
         if (i < nlr) {
-          const int ksteps = min(4, (p.r - 64 * i) / 16);
+          // packed: A k-steps [0, r/16) hold hi and [2, 2 + r/16) hold lo,
+          // both against B k-steps [0, r/16); unpacked: 4 k-steps per slot
+          const int ksteps = lr_packed ? p.r / 16 : 4;
           for (int kk = 0; kk < ksteps; ++kk) {
-            const uint64_t ad = make_sdesc(a0 + kk * 32, 16, 1024, kSwz128);
             const uint64_t bd = make_sdesc(b0 + kk * 32, 16, 1024, kSwz128);
-            umma_f16(tmem, ad, bd, id_f16, (i > 0 || kk > 0) ? 1u : 0u);
+            umma_f16(tmem, make_sdesc(a0 + kk * 32, 16, 1024, kSwz128), bd, id_f16,
+                     (i > 0 || kk > 0) ? 1u : 0u);
+            if (lr_packed)
+              umma_f16(tmem, make_sdesc(a0 + (2 + kk) * 32, 16, 1024, kSwz128), bd, id_f16, 1u);
           }
         } else {
           const uint32_t sa = smem_u32(stage_sfa(s));
@@ -211,17 +224,24 @@ __global__ void __launch_bounds__(kThreads, 1)
     const float gprod = __fmul_rn(gsa, gsw);
     const float alpha = __fdiv_rn(1.0f, gprod);
     if (nlr > 0) {
-      for (int c = 0; c < nlr; ++c) {
-        uint8_t* arow = stage_a(c % kStages) + row * 128;
+      // this row's xl·gs_a·gs_w split into bf16 hi + lo parts
+      for (int step = 0; step < nlr; ++step) {
+        uint8_t* arow = stage_a(step % kStages) + row * 128;
 #pragma unroll
         for (int j = 0; j < 8; ++j) {  // 8 bf16 = one 16-byte chunk
+          // packed: chunks 0-3 = hi of columns 0..31, chunks 4-7 = lo of them;
+          // unpacked: slice step/2, part step%2 (0 = hi, 1 = lo)
+          const int part = lr_packed ? (j >> 2) : (step & 1);
+          const int col0 = lr_packed ? 8 * (j & 3) : 64 * (step >> 1) + 8 * j;
           float v[8];
 #pragma unroll
           for (int e = 0; e < 8; ++e) {
-            const int col = 64 * c + 8 * j + e;
-            v[e] = (grow < p.M && col < p.r)
-                       ? __fmul_rn(p.lora[static_cast<size_t>(grow) * p.r + col], gprod)
-                       : 0.0f;
+            const int col = col0 + e;
+            float t = 0.0f;
+            if (grow < p.M && col < p.r)
+              t = __fmul_rn(p.lora[static_cast<size_t>(grow) * p.r + col], gprod);
+            const float hi = __bfloat162float(__float2bfloat16_rn(t));
+            v[e] = part == 0 ? hi : __fsub_rn(t, hi);
           }
           *reinterpret_cast<uint4*>(arow + ((j ^ (row & 7)) << 4)) =
               make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]),
