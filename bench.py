@@ -103,10 +103,11 @@ class ClockSampler:
 
 
 # ------------------------------------------------------- device workload --
-def make_sets(nsets, dev, seed_base=0):
-    """``nsets`` independent layers (weights + activations) prepared on the
-    device by the library's own offline prep; rotating through them keeps
-    every step's operands out of L2."""
+def make_sets(dev, l2_bytes):
+    """Independent copies of one layer (weights + activations + outputs),
+    prepared on the device by the library's own offline prep, enough of them
+    that their total exceeds 3x L2: rotating through them keeps every step's
+    operands out of L2."""
     import svdquant_w4a4_gemm_b200 as sv
     from svdquant_w4a4_gemm_b200 import prep as dprep
     d = workloads.draw_svdq(CASE)
@@ -115,30 +116,28 @@ def make_sets(nsets, dev, seed_base=0):
     b0 = torch.from_numpy(d["bias"]).to(dev).to(torch.bfloat16)
     xc = torch.from_numpy(d["x_cal"]).to(dev).to(torch.bfloat16)
     w0 = dprep.prepare_svdq(W0, b0, xc, CASE.r)
+    M, K, N, r = CASE.M, CASE.K, CASE.N, CASE.r
     gs = torch.empty(1, device=dev)
     sv.quantize_act(x0, w0.smooth, w0.L1t, None, out=(
-        torch.empty(CASE.M, CASE.K // 2, dtype=torch.uint8, device=dev),
-        torch.empty(sv.scale_bytes(CASE.M, CASE.K), dtype=torch.uint8, device=dev),
-        torch.empty(CASE.M, CASE.r, device=dev), gs))     # static scale from the data
+        torch.empty(M, K // 2, dtype=torch.uint8, device=dev),
+        torch.empty(sv.scale_bytes(M, K), dtype=torch.uint8, device=dev),
+        torch.empty(M, r, device=dev), gs))     # static activation scale from the data
+    per = (x0.numel() * 2 + M * K // 2 + sv.scale_bytes(M, K) + M * r * 4 + M * N * 2 +
+           w0.q_w.numel() + w0.sf_w.numel() + w0.L1t.numel() * 2 + w0.L2t.numel() * 2)
+    nsets = max(2, int(np.ceil(3 * l2_bytes / per)))
     sets = []
     for i in range(nsets):
         # distinct copies (same values) so that no two steps share memory
         w = sv.SvdqWeights(q_w=w0.q_w.clone(), sf_w=w0.sf_w.clone(), gs_w=w0.gs_w.clone(),
                            L1t=w0.L1t.clone(), L2t=w0.L2t.clone(), smooth=w0.smooth.clone(),
                            bias=w0.bias.clone())
-        M, K, N, r = CASE.M, CASE.K, CASE.N, CASE.r
         sets.append(dict(
             w=w, x=x0.clone(), gs=gs.clone(),
             q=torch.empty(M, K // 2, dtype=torch.uint8, device=dev),
             sf=torch.empty(sv.scale_bytes(M, K), dtype=torch.uint8, device=dev),
             lora=torch.empty(M, r, device=dev), gso=torch.empty(1, device=dev),
             y=torch.empty(M, N, dtype=torch.bfloat16, device=dev)))
-    return sets
-
-
-def set_bytes(s):
-    return sum(t.numel() * t.element_size() for t in
-               [s["x"], s["q"], s["sf"], s["lora"], s["y"], s["w"].q_w, s["w"].sf_w, s["w"].L1t, s["w"].L2t])
+    return sets, per
 
 
 def run_step(sv, s):
@@ -168,10 +167,8 @@ def bench_device(args, rank, world, dev):
     torch.cuda.set_device(dev)
     props = torch.cuda.get_device_properties(dev)
     l2 = getattr(props, "L2_cache_size", 126 * 2 ** 20) or 126 * 2 ** 20
-    probe = make_sets(1, dev)
-    per = set_bytes(probe[0])
-    nsets = max(2, int(np.ceil(3 * l2 / per)))
-    sets = probe + make_sets(nsets - 1, dev)[: nsets - 1]
+    sets, per = make_sets(dev, l2)
+    nsets = len(sets)
     stream = torch.cuda.current_stream(dev)
     M, K, N, r = CASE.M, CASE.K, CASE.N, CASE.r
 
@@ -179,8 +176,28 @@ def bench_device(args, rank, world, dev):
         run_step(sv, sets[i % nsets])
     sv.check_device_errors()
 
-    # ---- timed region: K steps, events around each kernel ----
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    # ---- the K timed steps, captured once into a CUDA graph so that the
+    # device time is not limited by host launch overhead; external timing
+    # events between the two kernels of every step give per-kernel times ----
+    ev = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(3)]
+          for _ in range(args.steps)]
+    graph = torch.cuda.CUDAGraph()
+    cap = torch.cuda.Stream(dev)
+    cap.wait_stream(stream)
+    with torch.cuda.graph(graph, stream=cap):
+        for i in range(args.steps):
+            s = sets[i % nsets]
+            e0, e1, e2 = ev[i]
+            e0.record()
+            sv.quantize_act(s["x"], s["w"].smooth, s["w"].L1t, s["gs"],
+                            out=(s["q"], s["sf"], s["lora"], s["gso"]))
+            e1.record()
+            sv.w4a4_linear(s["q"], s["sf"], s["gso"], s["lora"], s["w"], y=s["y"])
+            e2.record()
+    graph.replay()                      # untimed: uploads the graph
+    torch.cuda.synchronize(dev)
+    sv.check_device_errors()
+
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize(dev)
@@ -188,15 +205,7 @@ def bench_device(args, rank, world, dev):
     t_end = torch.cuda.Event(enable_timing=True)
     with ClockSampler(props_index(dev)) as clk:
         t_start.record(stream)
-        for i in range(args.steps):
-            s = sets[i % nsets]
-            e0, e1, e2 = ev[i]
-            e0.record(stream)
-            sv.quantize_act(s["x"], s["w"].smooth, s["w"].L1t, s["gs"],
-                            out=(s["q"], s["sf"], s["lora"], s["gso"]))
-            e1.record(stream)
-            sv.w4a4_linear(s["q"], s["sf"], s["gso"], s["lora"], s["w"], y=s["y"])
-            e2.record(stream)
+        graph.replay()
         t_end.record(stream)
         torch.cuda.synchronize(dev)
     if world > 1:
@@ -231,6 +240,7 @@ def bench_device(args, rank, world, dev):
     torch.cuda.synchronize(dev)
     e2e_ms = a.elapsed_time(b) / e2e_steps
 
+    del graph
     legs = bench_awq_legs(sv, dev, l2) if args.legs and rank == 0 else None
     return dict(total_ms=total_ms, k1_us=k1_us, k2_us=k2_us, clocks=clk.summary(), nsets=nsets,
                 set_mb=per / 2 ** 20, e2e_ms=e2e_ms, h2d=x_host.numel() * 2, d2h=y_host.numel() * 2,
