@@ -54,52 +54,65 @@ def peaks():
 
 # ------------------------------------------------------------------ clocks --
 class ClockSampler:
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    """Samples SM clock and clock-event reasons through NVML every 20 ms
+    while the timed region runs (the same counters nvidia-smi reports)."""
+    REASONS = {"sw_power_cap": 0x4, "hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20,
+               "hw_thermal_slowdown": 0x40, "hw_power_brake_slowdown": 0x80}
 
-    def __init__(self, gpu_index):
-        self.idx = gpu_index
-        self.proc = None
+    def __init__(self, dev):
+        self.dev = dev
+        self.samples = []
+        self.max_mhz = None
+        self._stop = None
+
+    def _handle(self):
+        import pynvml
+        pynvml.nvmlInit()
+        props = torch.cuda.get_device_properties(self.dev)
+        bus = getattr(props, "pci_bus_id", None)
+        if bus is not None:
+            dom = getattr(props, "pci_domain_id", 0)
+            devid = getattr(props, "pci_device_id", 0)
+            try:
+                return pynvml.nvmlDeviceGetHandleByPciBusId(f"{dom:08x}:{bus:02x}:{devid:02x}.0")
+            except pynvml.NVMLError:
+                pass
+        return pynvml.nvmlDeviceGetHandleByIndex(torch.device(self.dev).index or 0)
 
     def __enter__(self):
+        import threading
         try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "100"],
-                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-        except OSError:
-            self.proc = None
+            import pynvml
+            h = self._handle()
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            return self
+        self._stop = threading.Event()
+
+        def run():
+            get_reasons = getattr(pynvml, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                pynvml.nvmlDeviceGetCurrentClocksThrottleReasons
+            while not self._stop.is_set():
+                try:
+                    self.samples.append((pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM),
+                                         int(get_reasons(h))))
+                except Exception:
+                    pass
+                self._stop.wait(0.02)
+        self._t = threading.Thread(target=run, daemon=True)
+        self._t.start()
         return self
 
     def __exit__(self, *a):
-        self.lines = []
-        if self.proc is not None:
-            self.proc.terminate()
-            try:
-                out, _ = self.proc.communicate(timeout=5)
-            except subprocess.TimeoutExpired:
-                self.proc.kill()
-                out, _ = self.proc.communicate()
-            self.lines = [l for l in out.splitlines() if l.strip()]
+        if self._stop is not None:
+            self._stop.set()
+            self._t.join(timeout=2)
 
     def summary(self):
-        sm, mx, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for l in getattr(self, "lines", []):
-            f = [x.strip() for x in l.split(",")]
-            if len(f) < 9:
-                continue
-            try:
-                sm.append(float(f[1]))
-                mx = float(f[2])
-            except ValueError:
-                continue
-            for n, v in zip(names, f[5:9]):
-                if v.lower().startswith("active"):
-                    reasons.add(n)
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
-                "reasons": sorted(reasons), "samples": len(sm)}
+        sm = [c for c, _ in self.samples]
+        reasons = sorted({n for _, r in self.samples for n, b in self.REASONS.items() if r & b})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": self.max_mhz,
+                "reasons": reasons, "samples": len(sm)}
 
 
 # ------------------------------------------------------- device workload --
@@ -179,13 +192,15 @@ def bench_device(args, rank, world, dev):
     # ---- the K timed steps, captured once into a CUDA graph so that the
     # device time is not limited by host launch overhead; external timing
     # events between the two kernels of every step give per-kernel times ----
+    gsteps = min(args.steps, 200)                 # steps per captured graph
+    replays = max(1, -(-args.steps // gsteps))
     ev = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(3)]
-          for _ in range(args.steps)]
+          for _ in range(gsteps)]
     graph = torch.cuda.CUDAGraph()
     cap = torch.cuda.Stream(dev)
     cap.wait_stream(stream)
     with torch.cuda.graph(graph, stream=cap):
-        for i in range(args.steps):
+        for i in range(gsteps):
             s = sets[i % nsets]
             e0, e1, e2 = ev[i]
             e0.record()
@@ -203,9 +218,10 @@ def bench_device(args, rank, world, dev):
     torch.cuda.synchronize(dev)
     t_start = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)
-    with ClockSampler(props_index(dev)) as clk:
+    with ClockSampler(dev) as clk:
         t_start.record(stream)
-        graph.replay()
+        for _ in range(replays):
+            graph.replay()
         t_end.record(stream)
         torch.cuda.synchronize(dev)
     if world > 1:
@@ -216,6 +232,7 @@ def bench_device(args, rank, world, dev):
         t = torch.tensor([total_ms], device=dev)
         torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
         total_ms = float(t.item())
+    steps_done = gsteps * replays
     k1_us = [e[0].elapsed_time(e[1]) * 1e3 for e in ev]
     k2_us = [e[1].elapsed_time(e[2]) * 1e3 for e in ev]
 
@@ -242,7 +259,7 @@ def bench_device(args, rank, world, dev):
 
     del graph
     legs = bench_awq_legs(sv, dev, l2) if args.legs and rank == 0 else None
-    return dict(total_ms=total_ms, k1_us=k1_us, k2_us=k2_us, clocks=clk.summary(), nsets=nsets,
+    return dict(steps=steps_done, total_ms=total_ms, k1_us=k1_us, k2_us=k2_us, clocks=clk.summary(), nsets=nsets,
                 set_mb=per / 2 ** 20, e2e_ms=e2e_ms, h2d=x_host.numel() * 2, d2h=y_host.numel() * 2,
                 legs=legs)
 
@@ -360,7 +377,7 @@ def run_reference(args, rank, world):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--steps", type=int, default=20000)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--legs", action="store_true", help="also time the AWQ W4A16 modulation layer")
@@ -395,7 +412,8 @@ def main():
 
     M, K, N, r = CASE.M, CASE.K, CASE.N, CASE.r
     fl = layer_flops(M, K, N, r)
-    ms = res["total_ms"] / args.steps
+    steps = res["steps"]
+    ms = res["total_ms"] / steps
     value = fl * world / (ms * 1e-3) / 1e12
     pk = peaks()
     sustained = pk.get("bf16_tflops_sustained")
@@ -410,7 +428,7 @@ def main():
     k1_bytes = M * K * 2 + K * 4 + r * K * 2 + M * K // 2 + (M * K // 16) + M * r * 4
     hbm = pk.get("hbm_gbs", 6650.0)
     line = {
-        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": steps,
         "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "nvfp4", "data": "synthetic",
         "config": {"workload": WORKLOAD, "M": M, "K": K, "N": N, "r": r, "group": 16,
@@ -431,9 +449,10 @@ def main():
                                             "traffic": kernel_traffic("quantize.cu", "quantize_act_kernel")},
                     "w4a4_gemm_kernel": {"avg_launch_us": round(k2, 3)}},
         "clocks": res["clocks"],
+        "timed_region_ms": round(res["total_ms"], 3),
         "e2e": {"value": fl / (res["e2e_ms"] * 1e-3) / 1e12, "unit": UNIT,
                 "h2d_bytes_per_step": res["h2d"] + 4 * 0, "d2h_bytes_per_step": res["d2h"]},
-        "gpu_launches": 2 * args.steps,
+        "gpu_launches": 2 * steps,
         "cpu_baseline": cpu,
     }
     if res["legs"]:

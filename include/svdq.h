@@ -80,8 +80,8 @@ size_t svdq_nvfp4_scale_bytes(int64_t rows, int64_t K);
  *
  *   x_bf16      [M, K] bf16, row stride ldx elements (ldx >= K, ldx % 8 == 0).
  *   M, K        M >= 1, K >= 64, K % 64 == 0.
- *   smooth_s    [K] fp32 smoothing vector s (> 0).  The kernel multiplies x by
- *               RN_fp32(1/s_k).  NULL = no smoothing.
+ *   smooth_s    [K] fp32 smoothing vector s (> 0), 8-byte aligned.  The
+ *               kernel multiplies x by RN_fp32(1/s_k).  NULL = no smoothing.
  *   L1t_bf16    L1ᵀ, [r, K] bf16 row-major (K contiguous).  Ignored if r == 0.
  *   r           low-rank rank: 0 (no branch), 16, 32, 64 or 128.
  *   act_gscale  fp32 device scalar gs_a (static tensor scale).  NULL =
@@ -149,7 +149,7 @@ svdq_status svdq_w4a4_linear(const uint8_t* q_act, const uint8_t* sf_act,
  *   y[m,n] = bf16( Σ_k (x[m,k]·act_scale_inv[k]) · (q[n,k] − z[n,k/g])·sc[n,k/g] + b[n] )
  *
  *   x_bf16        [M, K] bf16, contiguous, 16-byte aligned.  1 <= M <= 8.
- *   K             K >= 64, K % 64 == 0; K <= 14464 for M <= 4 and K <= 7232
+ *   K             K >= 64, K % 64 == 0; K <= 14400 for M <= 4 and K <= 7104
  *                 for M > 4 (the per-CTA activation fragment table lives in
  *                 shared memory: 16 or 32 bytes per k).
  *   act_scale_inv [K] fp32 (1/a_k of the AWQ per-channel scale), 16-byte

@@ -255,7 +255,7 @@ svdq_status awq_w4a16_linear(const void* x_bf16, int64_t M, int64_t K, const flo
     return fail(SVDQ_ERR_INVALID_ARG, "x, qweight, scales, zeros and y must be non-null");
   if (M < 1 || M > 8) return fail(SVDQ_ERR_INVALID_ARG, "M=%lld must be in [1, 8]", (long long)M);
   if (group != 64) return fail(SVDQ_ERR_INVALID_ARG, "group=%d: only 64 is supported", group);
-  const int64_t kmax = M <= 4 ? 14464 : 7232;  // B-fragment table must fit in 227 KB of smem
+  const int64_t kmax = M <= 4 ? 14400 : 7104;  // B-fragment table must fit in 227 KB of smem
   if (K < 64 || K % 64 != 0 || K > kmax)
     return fail(SVDQ_ERR_INVALID_ARG, "K=%lld must be a multiple of 64 in [64, %lld] for M=%lld",
                 (long long)K, (long long)kmax, (long long)M);

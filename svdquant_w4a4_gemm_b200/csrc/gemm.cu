@@ -3,34 +3,35 @@
 // 4-bit compute kernel", blog.margrop.com "技术细节 §1", SVDQuant step 4).
 //
 //   y = bf16( α·acc + bias ),  α = 1/(gs_a·gs_w)
-//   acc = (hi + lo)·L2                      (kind::f16 MMAs, first)
-//       + Σ_k e2m1_a·sfa · e2m1_w·sfw      (kind::mxf4nvf4 block-scaled MMAs)
+//   acc = Σ_k e2m1_a·sfa · e2m1_w·sfw      (kind::mxf4nvf4 block-scaled MMAs)
+//       + (hi + lo)·L2                      (kind::f16 MMAs, same accumulator)
 //   hi = bf16(xl·gs_a·gs_w), lo = bf16(xl·gs_a·gs_w − hi)
 // The low-rank term can dominate y (it carries the outlier channels), so
 // its activation operand keeps ~16 significant bits through the hi/lo
 // split; L2 itself is bf16 by construction.
 //
-// One CTA computes a 128 x BN tile of y (BN = 256, or 128 when N is not a
-// multiple of 256), fp32 accumulator in tensor memory (TMEM).
-//   warp 0     producer: TMA loads of the packed FP4 operands (128-byte rows,
-//              128-byte swizzle: 16 KB of A and BN x 128 B of B per stage,
-//              256 K-elements), plain bulk copies of the matching scale
-//              blocks (the 128x4 block layout is already the byte order the
-//              scale copy to TMEM wants: 2 KB per 128 rows per stage), and
-//              TMA loads of L2ᵀ for the low-rank steps.
-//   warp 1     TMEM owner and MMA issuer (one thread): per stage it copies
-//              the stage's scale blocks smem -> TMEM (tcgen05.cp 32x128b
-//              .warpx4, 4 columns per 128 rows per 64 K) and issues four
-//              block-scaled MMAs (K = 64 each); tcgen05.commit frees the stage.
-//   warps 2-5  first convert the [128 x r] fp32 down-projection rows into
-//              the hi/lo bf16 parts in the A slot of the first ring stages
-//              (128-byte swizzle written by hand), then run the epilogue:
-//              TMEM -> registers, α·acc + bias, bf16, store.
-// The low-rank steps go through the same shared-memory ring as the FP4
-// stages, so they need no memory of their own: for r <= 32 one ring slot
-// holds hi in A columns [0, 32) and lo in [32, 64) against one L2ᵀ slice;
-// for r = 64, 128 each 64-wide slice of r takes two slots (hi, then lo),
-// both loading the same L2ᵀ slice.
+// Persistent kernel: one CTA per SM walks 128 x BN output tiles (BN = 256,
+// or 128 when N is not a multiple of 256); fp32 accumulator in TMEM.
+//   warp 0     producer.  For each tile: the FP4 steps (TMA of 128-byte rows
+//              of packed A and B = 256 K-elements, 128-byte swizzle; bulk
+//              copies of the matching scale blocks — the 128x4 block layout
+//              is already the byte order the scale copy to TMEM wants),
+//              then the low-rank steps (TMA of a 64-wide slice of L2ᵀ).
+//              All go through one kStages-deep shared-memory ring.
+//   warp 1     TMEM owner and MMA issuer (one thread).  Per FP4 step:
+//              tcgen05.cp of the scale blocks into TMEM (4 columns per 128
+//              rows per 64 K), four block-scaled MMAs (K = 64 each).  Per
+//              low-rank step: kind::f16 MMAs into the same accumulator.
+//              tcgen05.commit frees ring slots and, after a tile's last
+//              step, hands the accumulator to the epilogue.
+//   warps 2-9  epilogue, two warps per 32-lane TMEM quadrant (one per half
+//              of BN).  During a tile's mainloop they write the tile's
+//              low-rank A operand (hi/lo bf16 of the fp32 down-projection,
+//              swizzled by hand) into the ring slots of its low-rank steps
+//              and stage the bias slice in shared memory; after the
+//              accumulator is full they drain TMEM -> registers (α·acc +
+//              bias -> bf16), release the accumulator to the MMA warp and
+//              store y while the next tile's mainloop runs.
 #include "internal.h"
 #include "ptx.cuh"
 
@@ -38,13 +39,15 @@ namespace svdq {
 namespace {
 
 constexpr int kBM = 128;
-constexpr int kBKBytes = 128;  // 256 FP4 elements per stage and row
+constexpr int kBKBytes = 128;  // 256 FP4 elements per FP4 step and row
 constexpr int kStages = 4;
-constexpr int kThreads = 192;
+constexpr int kEpiWarps = 8;
+constexpr int kThreads = 32 * (2 + kEpiWarps);
 constexpr uint32_t kATileBytes = kBM * kBKBytes;  // 16 KB
 
 struct GemmParams {
-  int M, N, K, r, bn;
+  int M, N, K, r;
+  int tiles_n, tiles;     // output tiles along N, total
   const uint8_t* sf_a;
   const uint8_t* sf_w;
   const float* gs_a;
@@ -53,7 +56,7 @@ struct GemmParams {
   const uint16_t* bias;   // [N] or null
   uint16_t* y;
   int64_t ldy;
-  int fault;              // test hook: 1 = skip the first stage's loads
+  int fault;              // test hook: 1 = the first ring slot never fills
   WaitCfg wait;
 };
 
@@ -68,12 +71,21 @@ struct Layout {
   static constexpr uint32_t kSfa = 4 * 512;              // 4 K-blocks x 128 rows
   static constexpr uint32_t kSfb = (BN / 128) * 4 * 512;
   static constexpr uint32_t kStage = kATileBytes + kB + kSfa + kSfb;
-  static constexpr uint32_t kTmemCols = 512;             // acc BN + scales
+  static constexpr uint32_t kRing = kStages * kStage;
+  static constexpr uint32_t kBias = kEpiWarps * (BN / 2) * 2;  // per-warp bias slices
+  static constexpr uint32_t kTmemCols = BN == 256 ? 512 : 256;
   static constexpr uint32_t kSfaCol = BN;                // 16 columns
   static constexpr uint32_t kSfbCol = BN + 16;           // (BN/128)*16 columns
+  static constexpr int kColsPerWarp = BN / 2;            // epilogue columns per warp
   static_assert(kStage % 1024 == 0, "stage must keep 1 KB alignment");
-  static_assert(BN + 16 + (BN / 128) * 16 <= 512, "TMEM budget");
+  static_assert(BN + 16 + (BN / 128) * 16 <= kTmemCols, "TMEM budget");
 };
+
+// Where tile `t` sits in the output.
+__device__ __forceinline__ void tile_coords(int t, int tiles_n, int bn, int& m0, int& n0) {
+  m0 = (t / tiles_n) * kBM;
+  n0 = (t % tiles_n) * bn;
+}
 
 template <int BN>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -84,33 +96,34 @@ __global__ void __launch_bounds__(kThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
-  uint64_t* full = reinterpret_cast<uint64_t*>(base + kStages * L::kStage);
+  uint16_t* bias_s = reinterpret_cast<uint16_t*>(base + L::kRing);
+  uint64_t* full = reinterpret_cast<uint64_t*>(base + L::kRing + L::kBias);
   uint64_t* empty = full + kStages;
-  uint64_t* lr_full = empty + kStages;
-  uint64_t* acc_full = lr_full + 1;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_full + 1);
+  uint64_t* lrf = empty + kStages;       // low-rank A written, per ring slot
+  uint64_t* acc_full = lrf + kStages;
+  uint64_t* acc_empty = acc_full + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 1);
   auto stage_a = [&](int s) { return base + s * L::kStage; };
   auto stage_b = [&](int s) { return base + s * L::kStage + kATileBytes; };
   auto stage_sfa = [&](int s) { return base + s * L::kStage + kATileBytes + L::kB; };
   auto stage_sfb = [&](int s) { return base + s * L::kStage + kATileBytes + L::kB + L::kSfa; };
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int n0 = blockIdx.x * BN;
-  const int m0 = blockIdx.y * kBM;
   const bool lr_packed = p.r > 0 && p.r <= 32;  // hi and lo share one A tile
-  const int nlr = p.r == 0 ? 0 : (lr_packed ? 1 : 2 * (p.r / 64));  // low-rank ring steps
+  const int nlr = p.r == 0 ? 0 : (lr_packed ? 1 : 2 * (p.r / 64));  // low-rank steps per tile
   const int kblocks = p.K / 64;              // 64-element K blocks (one MMA each)
-  const int nk = (kblocks + 3) / 4;          // FP4 ring steps (256 K each, last may be short)
-  const int nsteps = nlr + nk;
+  const int nk = (kblocks + 3) / 4;          // FP4 steps per tile (last may be short)
+  const int nsteps = nk + nlr;               // ring steps per tile
   const int nb_total = (p.N + 127) / 128;    // 128-row blocks of the weight scales
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
+      mbar_init(&lrf[s], kEpiWarps / 2);
     }
-    mbar_init(lr_full, 4);
     mbar_init(acc_full, 1);
+    mbar_init(acc_empty, kEpiWarps);
     fence_mbar_init();
   }
   if (warp == 0 && lane == 0) {
@@ -130,35 +143,46 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0) {
     // ------------------------------------------------------- producer ----
     if (lane == 0) {
-      int issued = 0;
-      for (int i = 0; i < nsteps; ++i) {
-        const int s = i % kStages;
-        const uint32_t ph = (i / kStages) & 1;
-        if (!mbar_wait(&empty[s], ph ^ 1, p.wait, kErrTimeoutEmpty)) break;
-        if (p.fault == 1 && i == 0) continue;  // test hook: this stage never fills
-        if (i < nlr) {
-          // L2ᵀ[n0 .. n0+BN) x r[64c .. 64c+64) as bf16, zero-filled past r
-          const int c = lr_packed ? 0 : i / 2;
-          mbar_arrive_expect_tx(&full[s], L::kB);
-          tma_load_2d(stage_b(s), &tmap_l2, &full[s], 64 * c, n0);
-        } else {
-          const int kb = i - nlr;  // 256-element K step
-          const int nkb = min(4, kblocks - 4 * kb);                  // scale blocks (MMAs) in it
-          const int nbl = min(BN / 128, nb_total - n0 / 128);        // weight scale row blocks
-          const uint32_t sfbytes = static_cast<uint32_t>(nkb) * 512;
-          mbar_arrive_expect_tx(&full[s], kATileBytes + L::kB + sfbytes * (1 + nbl));
-          tma_load_2d(stage_a(s), &tmap_a, &full[s], kb * kBKBytes, m0);
-          tma_load_2d(stage_b(s), &tmap_b, &full[s], kb * kBKBytes, n0);
-          bulk_load(stage_sfa(s), p.sf_a + (static_cast<size_t>(m0 / 128) * kblocks + 4 * kb) * 512,
-                    sfbytes, &full[s]);
-          for (int nb = 0; nb < nbl; ++nb)
-            bulk_load(stage_sfb(s) + nb * 2048,
-                      p.sf_w + (static_cast<size_t>(n0 / 128 + nb) * kblocks + 4 * kb) * 512,
+      int it = 0;          // ring step counter (continues across tiles)
+      int issued_to = 0;   // ring steps whose loads were issued
+      bool ok = true;
+      for (int t = blockIdx.x; ok && t < p.tiles; t += gridDim.x) {
+        int m0, n0;
+        tile_coords(t, p.tiles_n, BN, m0, n0);
+        const int nbl = min(BN / 128, nb_total - n0 / 128);  // weight scale row blocks
+        for (int st = 0; st < nsteps; ++st, ++it) {
+          const int s = it % kStages;
+          const uint32_t ph = (it / kStages) & 1;
+          if (!mbar_wait(&empty[s], ph ^ 1, p.wait, kErrTimeoutEmpty)) {
+            ok = false;
+            break;
+          }
+          if (st < nk) {
+            if (p.fault == 1 && it == 0) continue;  // test hook: this slot never fills
+            const int kb = st;                      // 256-element K step
+            const int nkb = min(4, kblocks - 4 * kb);
+            const uint32_t sfbytes = static_cast<uint32_t>(nkb) * 512;
+            mbar_arrive_expect_tx(&full[s], kATileBytes + L::kB + sfbytes * (1 + nbl));
+            tma_load_2d(stage_a(s), &tmap_a, &full[s], kb * kBKBytes, m0);
+            tma_load_2d(stage_b(s), &tmap_b, &full[s], kb * kBKBytes, n0);
+            bulk_load(stage_sfa(s), p.sf_a + (static_cast<size_t>(m0 / 128) * kblocks + 4 * kb) * 512,
                       sfbytes, &full[s]);
+            for (int nb = 0; nb < nbl; ++nb)
+              bulk_load(stage_sfb(s) + nb * 2048,
+                        p.sf_w + (static_cast<size_t>(n0 / 128 + nb) * kblocks + 4 * kb) * 512,
+                        sfbytes, &full[s]);
+          } else {
+            // L2ᵀ[n0 .. n0+BN) x r[64c .. 64c+64) as bf16, zero-filled past r
+            const int j = st - nk;
+            const int c = lr_packed ? 0 : j / 2;
+            mbar_arrive_expect_tx(&full[s], L::kB);
+            tma_load_2d(stage_b(s), &tmap_l2, &full[s], 64 * c, n0);
+          }
+          issued_to = it + 1;
         }
-        issued = i + 1;
       }
-      for (int i = max(0, issued - kStages); i < issued; ++i) {
+      // never leave the CTA with a copy still landing in its shared memory
+      for (int i = max(0, issued_to - kStages); i < issued_to; ++i) {
         if (p.fault == 1 && i == 0) continue;
         mbar_wait(&full[i % kStages], (i / kStages) & 1, p.wait, kErrTimeoutDrain);
       }
@@ -168,111 +192,177 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       const uint32_t id_f16 = idesc_f16(128, BN, true);
       const uint32_t id_fp4 = idesc_nvfp4(128, BN);
+      int it = 0;
+      uint32_t lr_par = 0;                   // parity of each slot's next low-rank phase
+      int local = 0;                         // tiles done by this CTA
       bool ok = true;
-      if (nlr > 0 && !mbar_wait(lr_full, 0, p.wait, kErrTimeoutFull)) ok = false;
-      tc_fence_after();
-      for (int i = 0; ok && i < nsteps; ++i) {
-        const int s = i % kStages;
-        const uint32_t ph = (i / kStages) & 1;
-        if (!mbar_wait(&full[s], ph, p.wait, kErrTimeoutFull)) {
+      for (int t = blockIdx.x; ok && t < p.tiles; t += gridDim.x, ++local) {
+        // the epilogue must have drained the previous tile's accumulator
+        if (local > 0 && !mbar_wait(acc_empty, (local - 1) & 1, p.wait, kErrTimeoutAcc)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        const uint32_t a0 = smem_u32(stage_a(s));
-        const uint32_t b0 = smem_u32(stage_b(s));
-        if (i < nlr) {
-          // packed: A k-steps [0, r/16) hold hi and [2, 2 + r/16) hold lo,
-          // both against B k-steps [0, r/16); unpacked: 4 k-steps per slot
-          const int ksteps = lr_packed ? p.r / 16 : 4;
-          for (int kk = 0; kk < ksteps; ++kk) {
-            const uint64_t bd = make_sdesc(b0 + kk * 32, 16, 1024, kSwz128);
-            umma_f16(tmem, make_sdesc(a0 + kk * 32, 16, 1024, kSwz128), bd, id_f16,
-                     (i > 0 || kk > 0) ? 1u : 0u);
-            if (lr_packed)
-              umma_f16(tmem, make_sdesc(a0 + (2 + kk) * 32, 16, 1024, kSwz128), bd, id_f16, 1u);
+        for (int st = 0; st < nsteps; ++st, ++it) {
+          const int s = it % kStages;
+          const uint32_t ph = (it / kStages) & 1;
+          if (!mbar_wait(&full[s], ph, p.wait, kErrTimeoutFull)) {
+            ok = false;
+            break;
           }
-        } else {
-          const uint32_t sa = smem_u32(stage_sfa(s));
-          const uint32_t sb = smem_u32(stage_sfb(s));
-          const int nkb = min(4, kblocks - 4 * (i - nlr));
-          for (int kk = 0; kk < nkb; ++kk) {
-            tmem_cp_32x128b_warpx4(tmem + L::kSfaCol + 4 * kk, make_sdesc(sa + kk * 512, 128, 128, kSwzNone));
+          const uint32_t a0 = smem_u32(stage_a(s));
+          const uint32_t b0 = smem_u32(stage_b(s));
+          if (st < nk) {
+            tc_fence_after();
+            const uint32_t sa = smem_u32(stage_sfa(s));
+            const uint32_t sb = smem_u32(stage_sfb(s));
+            const int nkb = min(4, kblocks - 4 * st);
+            for (int kk = 0; kk < nkb; ++kk) {
+              tmem_cp_32x128b_warpx4(tmem + L::kSfaCol + 4 * kk,
+                                     make_sdesc(sa + kk * 512, 128, 128, kSwzNone));
 #pragma unroll
-            for (int nb = 0; nb < BN / 128; ++nb)
-              tmem_cp_32x128b_warpx4(tmem + L::kSfbCol + (BN / 128) * 4 * kk + 4 * nb,
-                                     make_sdesc(sb + (nb * 4 + kk) * 512, 128, 128, kSwzNone));
+              for (int nb = 0; nb < BN / 128; ++nb)
+                tmem_cp_32x128b_warpx4(tmem + L::kSfbCol + (BN / 128) * 4 * kk + 4 * nb,
+                                       make_sdesc(sb + (nb * 4 + kk) * 512, 128, 128, kSwzNone));
+            }
+            for (int kk = 0; kk < nkb; ++kk) {
+              const uint64_t ad = make_sdesc(a0 + kk * 32, 16, 1024, kSwz128);
+              const uint64_t bd = make_sdesc(b0 + kk * 32, 16, 1024, kSwz128);
+              umma_nvfp4(tmem, ad, bd, id_fp4, tmem + L::kSfaCol + 4 * kk,
+                         tmem + L::kSfbCol + (BN / 128) * 4 * kk, (st > 0 || kk > 0) ? 1u : 0u);
+            }
+          } else {
+            if (!mbar_wait(&lrf[s], (lr_par >> s) & 1u, p.wait, kErrTimeoutFull)) {
+              ok = false;
+              break;
+            }
+            lr_par ^= 1u << s;
+            tc_fence_after();
+            // packed: A k-steps [0, r/16) hold hi and [2, 2 + r/16) hold lo,
+            // both against B k-steps [0, r/16); unpacked: 4 k-steps per slot
+            const int ksteps = lr_packed ? p.r / 16 : 4;
+            for (int kk = 0; kk < ksteps; ++kk) {
+              const uint64_t bd = make_sdesc(b0 + kk * 32, 16, 1024, kSwz128);
+              umma_f16(tmem, make_sdesc(a0 + kk * 32, 16, 1024, kSwz128), bd, id_f16, 1u);
+              if (lr_packed)
+                umma_f16(tmem, make_sdesc(a0 + (2 + kk) * 32, 16, 1024, kSwz128), bd, id_f16, 1u);
+            }
           }
-          for (int kk = 0; kk < nkb; ++kk) {
-            const uint64_t ad = make_sdesc(a0 + kk * 32, 16, 1024, kSwz128);
-            const uint64_t bd = make_sdesc(b0 + kk * 32, 16, 1024, kSwz128);
-            umma_nvfp4(tmem, ad, bd, id_fp4, tmem + L::kSfaCol + 4 * kk,
-                       tmem + L::kSfbCol + (BN / 128) * 4 * kk,
-                       (i > 0 || kk > 0) ? 1u : 0u);
-          }
+          umma_commit(&empty[s]);
         }
-        umma_commit(&empty[s]);
+        if (ok) umma_commit(acc_full);
       }
-      if (ok) umma_commit(acc_full);
     }
   } else {
-    // --------------------------------------- low-rank A, then epilogue ----
-    const int quad = warp & 3;
-    const int row = 32 * quad + lane;  // TMEM lane == tile row
-    const int grow = m0 + row;
-    const float gsa = *p.gs_a, gsw = *p.gs_w;
-    const float gprod = __fmul_rn(gsa, gsw);
+    // ---------------------------------------------------------- epilogue ----
+    const int ew = warp - 2;                 // 0..7
+    const int quad = warp & 3;               // TMEM lane quadrant this warp may access
+    const int half = ew >> 2;                // which half of BN
+    const int row = 32 * quad + lane;        // tile row == TMEM lane
+    const float gprod = __fmul_rn(*p.gs_a, *p.gs_w);
     const float alpha = __fdiv_rn(1.0f, gprod);
-    if (nlr > 0) {
-      // this row's xl·gs_a·gs_w split into bf16 hi + lo parts
-      for (int step = 0; step < nlr; ++step) {
-        uint8_t* arow = stage_a(step % kStages) + row * 128;
+    constexpr int kCols = L::kColsPerWarp;
+    int it = 0;
+    int local = 0;
+    bool ok = true;
+    for (int t = blockIdx.x; ok && t < p.tiles; t += gridDim.x, ++local) {
+      int m0, n0;
+      tile_coords(t, p.tiles_n, BN, m0, n0);
+      const int grow = m0 + row;
+      // (1) this warp's bias slice into its own shared-memory buffer (only
+      // this warp reads it, after the __syncwarp below, and it rewrites it
+      // only after its previous drain finished reading it)
+      uint16_t* bsl = bias_s + ew * kCols;
+      for (int c = lane; c < kCols; c += 32) {
+        const int col = n0 + half * kCols + c;
+        bsl[c] = (p.bias && col < p.N) ? p.bias[col] : static_cast<uint16_t>(0);
+      }
+      __syncwarp();
+      // (2) the low-rank A operand of this tile, into the ring slots of its
+      // low-rank steps (they follow the tile's FP4 steps); one warp per
+      // quadrant writes its 32 rows
+      it += nk;
+      for (int j = 0; j < nlr; ++j, ++it) {
+        const int s = it % kStages;
+        const uint32_t ph = (it / kStages) & 1;
+        if (half != 0) continue;
+        if (!mbar_wait(&empty[s], ph ^ 1, p.wait, kErrTimeoutEmpty)) {
+          ok = false;
+          break;
+        }
+        uint8_t* arow = stage_a(s) + row * 128;
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {  // 8 bf16 = one 16-byte chunk
+        for (int q = 0; q < 8; ++q) {  // 8 bf16 = one 16-byte chunk
           // packed: chunks 0-3 = hi of columns 0..31, chunks 4-7 = lo of them;
-          // unpacked: slice step/2, part step%2 (0 = hi, 1 = lo)
-          const int part = lr_packed ? (j >> 2) : (step & 1);
-          const int col0 = lr_packed ? 8 * (j & 3) : 64 * (step >> 1) + 8 * j;
+          // unpacked: slice j/2, part j%2 (0 = hi, 1 = lo)
+          const int part = lr_packed ? (q >> 2) : (j & 1);
+          const int col0 = lr_packed ? 8 * (q & 3) : 64 * (j >> 1) + 8 * q;
           float v[8];
+          if (grow < p.M && col0 < p.r) {
+            const float4* src =
+                reinterpret_cast<const float4*>(p.lora + static_cast<size_t>(grow) * p.r + col0);
+            const float4 u0 = src[0], u1 = src[1];
+            const float w8[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
 #pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            const int col = col0 + e;
-            float t = 0.0f;
-            if (grow < p.M && col < p.r)
-              t = __fmul_rn(p.lora[static_cast<size_t>(grow) * p.r + col], gprod);
-            const float hi = __bfloat162float(__float2bfloat16_rn(t));
-            v[e] = part == 0 ? hi : __fsub_rn(t, hi);
+            for (int e = 0; e < 8; ++e) {
+              const float tv = __fmul_rn(w8[e], gprod);
+              const float hi = __bfloat162float(__float2bfloat16_rn(tv));
+              v[e] = part == 0 ? hi : __fsub_rn(tv, hi);
+            }
+          } else {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) v[e] = 0.0f;
           }
-          *reinterpret_cast<uint4*>(arow + ((j ^ (row & 7)) << 4)) =
+          *reinterpret_cast<uint4*>(arow + ((q ^ (row & 7)) << 4)) =
               make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]),
                          pack_bf16x2(v[4], v[5]), pack_bf16x2(v[6], v[7]));
         }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&lrf[s]);
       }
-      fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(lr_full);
-    }
-    if (mbar_wait(acc_full, 0, p.wait, kErrTimeoutAcc)) {
+      if (!ok) break;
+      // (3) drain the accumulator: α·acc + bias -> packed bf16 in registers
+      if (!mbar_wait(acc_full, local & 1, p.wait, kErrTimeoutAcc)) {
+        ok = false;
+        break;
+      }
       tc_fence_after();
-#pragma unroll 1
-      for (int c = 0; c < BN / 16; ++c) {
-        uint32_t acc[16];
-        tmem_ld_32x32b_x16(tmem + (static_cast<uint32_t>(32 * quad) << 16) + c * 16, acc);
-        tmem_ld_wait();
-        const int col = n0 + c * 16;
-        if (grow < p.M && col < p.N) {
-          float o[16];
+      uint32_t packed[kCols / 2];
+      const uint32_t taddr = tmem + (static_cast<uint32_t>(32 * quad) << 16) + half * kCols;
 #pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            const float b = p.bias ? __uint_as_float(static_cast<uint32_t>(p.bias[col + e]) << 16) : 0.0f;
-            o[e] = __fadd_rn(__fmul_rn(__uint_as_float(acc[e]), alpha), b);
+      for (int c = 0; c < kCols / 16; c += 2) {
+        uint32_t a0[16], a1[16];
+        tmem_ld_32x32b_x16(taddr + c * 16, a0);
+        tmem_ld_32x32b_x16(taddr + (c + 1) * 16, a1);
+        tmem_ld_wait();
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+          const uint32_t* a = u ? a1 : a0;
+          const uint4* b4 = reinterpret_cast<const uint4*>(bsl + (c + u) * 16);
+          const uint4 bb0 = b4[0], bb1 = b4[1];
+          const uint32_t bw[8] = {bb0.x, bb0.y, bb0.z, bb0.w, bb1.x, bb1.y, bb1.z, bb1.w};
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const float lo = __fadd_rn(__fmul_rn(__uint_as_float(a[2 * e]), alpha),
+                                       __uint_as_float(bw[e] << 16));
+            const float hi = __fadd_rn(__fmul_rn(__uint_as_float(a[2 * e + 1]), alpha),
+                                       __uint_as_float(bw[e] & 0xFFFF0000u));
+            packed[(c + u) * 8 + e] = pack_bf16x2(lo, hi);
           }
-          uint4* dst = reinterpret_cast<uint4*>(p.y + static_cast<size_t>(grow) * p.ldy + col);
-          dst[0] = make_uint4(pack_bf16x2(o[0], o[1]), pack_bf16x2(o[2], o[3]),
-                              pack_bf16x2(o[4], o[5]), pack_bf16x2(o[6], o[7]));
-          dst[1] = make_uint4(pack_bf16x2(o[8], o[9]), pack_bf16x2(o[10], o[11]),
-                              pack_bf16x2(o[12], o[13]), pack_bf16x2(o[14], o[15]));
         }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(acc_empty);   // the MMA may start the next tile
+      // (4) store y (overlaps the next tile's mainloop)
+      const int colb = n0 + half * kCols;
+      if (grow < p.M) {
+        uint4* dst = reinterpret_cast<uint4*>(p.y + static_cast<size_t>(grow) * p.ldy + colb);
+#pragma unroll
+        for (int q = 0; q < kCols / 8; ++q)
+          if (colb + 8 * q < p.N)
+            dst[q] = make_uint4(packed[4 * q], packed[4 * q + 1], packed[4 * q + 2], packed[4 * q + 3]);
       }
     }
   }
@@ -286,16 +376,18 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 template <int BN>
 svdq_status launch_bn(const LaunchCtx& ctx, const CUtensorMap& ta, const CUtensorMap& tb,
-                      const CUtensorMap& tl, const GemmParams& p) {
+                      const CUtensorMap& tl, GemmParams p) {
   using L = Layout<BN>;
-  const size_t smem = 1024 + kStages * static_cast<size_t>(L::kStage) + 8 * (2 * kStages + 2) + 16;
+  const size_t smem = 1024 + static_cast<size_t>(L::kRing) + L::kBias + 8 * (3 * kStages + 2) + 16;
   static bool attr_done[64] = {};
   if (!attr_done[ctx.device & 63]) {
     cudaFuncSetAttribute(w4a4_gemm_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          static_cast<int>(smem));
     attr_done[ctx.device & 63] = true;
   }
-  dim3 grid((p.N + BN - 1) / BN, (p.M + kBM - 1) / kBM);
+  p.tiles_n = (p.N + BN - 1) / BN;
+  p.tiles = p.tiles_n * ((p.M + kBM - 1) / kBM);
+  const int grid = std::min(p.tiles, ctx.num_sms);
   w4a4_gemm_kernel<BN><<<grid, kThreads, smem, ctx.stream>>>(ta, tb, tl, p);
   return check_launch("w4a4_gemm_kernel");
 }
@@ -315,8 +407,8 @@ svdq_status launch_w4a4_gemm(const LaunchCtx& ctx, const uint8_t* q_act, const u
   if (!make_tmap_2d(&tb, q_w, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, N, K / 2, K / 2, bn, kBKBytes, 128))
     return SVDQ_ERR_CUDA;
   if (r > 0) {
-    if (!make_tmap_2d(&tl, L2t, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, N, r, static_cast<uint64_t>(r) * 2,
-                      bn, 64, 128))
+    if (!make_tmap_2d(&tl, L2t, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, N, r,
+                      static_cast<uint64_t>(r) * 2, bn, 64, 128))
       return SVDQ_ERR_CUDA;
   } else {
     tl = ta;
@@ -326,7 +418,6 @@ svdq_status launch_w4a4_gemm(const LaunchCtx& ctx, const uint8_t* q_act, const u
   p.N = static_cast<int>(N);
   p.K = static_cast<int>(K);
   p.r = r;
-  p.bn = bn;
   p.sf_a = sf_act;
   p.sf_w = sf_w;
   p.gs_a = act_gscale;

@@ -6,23 +6,30 @@
 // ("Bringing Nunchaku 4-bit Diffusion Inference to Diffusers", as told on
 // blog.margrop.com "技术细节 §1", SVDQuant step 4).
 //
-// Design (one CTA = 128 rows x kc columns of x; kc % 64 == 0):
-//   warp 0      TMA producer: streams 128x64 bf16 tiles of x (128-byte
-//               swizzle, 16 KB) and the matching 64-column slice of L1ᵀ
-//               into a kStages-deep shared-memory ring (mbarrier tx counts).
-//   warp 1      owns tensor memory; one thread issues the tcgen05 kind::f16
-//               MMAs of the down-projection: D[128 x r] += bf16(x̂)[128x64] ·
-//               L1ᵀ[r x 64]ᵀ, fp32 accumulator in TMEM.
-//   warps 2-9   quantizers: each thread takes one row and 32 columns of the
-//               tile (two 16-element groups): x̂ = x·inv_s, group max, E4M3
-//               scale, E2M1 codes (hardware cvt, round-to-nearest-even,
-//               satfinite), 16-byte code store, 2-byte scale store into the
-//               128x4 block layout, and writes bf16(x̂) back over x in
-//               shared memory for the MMA.  At the end they read the
-//               accumulator from TMEM and add it into lora_out (the K range
-//               is split over CTAs to fill the GPU, so partial sums meet with
-//               vector atomics in L2; lora_out is zeroed first).
-// HBM traffic is the algorithmic minimum: x once, codes + scales + x̂·L1 once;
+// Work unit: a 128-row x 64-column sub-tile of x (16 KB of bf16, one
+// 128-byte-swizzled TMA box).  The ceil(M/128)·(K/64) sub-tiles, in
+// row-block-major order, are split into one contiguous, equal range per CTA
+// (one persistent CTA per SM), so the memory pipeline never drains between
+// work items and the load is balanced to one sub-tile.
+//   warp 0       TMA producer: x sub-tiles and the matching 64-column slices
+//                of L1ᵀ into a kStages-deep shared-memory ring; its lanes
+//                also compute RN(1/s) for the slot's 64 columns.
+//   warp 1       TMEM owner; one thread issues the down-projection as
+//                tcgen05 kind::f16 MMAs (M = 128, N = r, K = 16 each) from
+//                the quantized tile's bf16(x̂) and the L1ᵀ slice into a TMEM
+//                accumulator; a new accumulator (of two) per run of
+//                sub-tiles in the same 128-row block ("segment").
+//   warps 2-9    quantizers: one thread = one row x 32 columns = two
+//                16-element groups: x̂ = x·inv_s, group max, E4M3 scale
+//                (cvt.rn.satfinite.e4m3x2), E2M1 codes (cvt.rn.satfinite
+//                .e2m1x2, sign bit copied), a 16-byte code store, a 2-byte
+//                scale store into the 128x4 block layout, and bf16(x̂)
+//                written back over the tile for the MMA.
+//   warps 10-13  epilogue: when a segment's accumulator is complete, TMEM ->
+//                registers -> float4 atomics into xl (zeroed beforehand:
+//                a row block's K range can span several CTAs), then release
+//                the accumulator.
+// HBM traffic is the algorithmic minimum: x once, codes + scales + xl once;
 // L1ᵀ slices come from L2.
 #include <cstdio>
 
@@ -36,11 +43,13 @@ constexpr int kBM = 128;
 constexpr int kSubK = 64;
 constexpr int kStages = 4;
 constexpr int kQuantWarps = 8;
-constexpr int kThreads = 32 * (2 + kQuantWarps);
+constexpr int kEpiWarps = 4;
+constexpr int kThreads = 32 * (2 + kQuantWarps + kEpiWarps);
 constexpr uint32_t kXTileBytes = kBM * kSubK * 2;
 
 struct QuantParams {
-  int M, K, r, kc;
+  int M, K, r;
+  int units;              // ceil(M/128) * (K/64) sub-tiles
   const float* smooth_s;  // [K] or null
   const float* gs_in;     // static tensor scale, or null for dynamic
   const float* amax_src;  // dynamic: amax bits (written by the amax pass)
@@ -72,6 +81,12 @@ __device__ __forceinline__ float tensor_scale_from_amax(float amax) {
   return amax > 0.0f ? __fdiv_rn(2688.0f, amax) : 1.0f;
 }
 
+// This CTA's contiguous range of sub-tiles.
+__device__ __forceinline__ void unit_range(int units, int& u0, int& u1) {
+  u0 = static_cast<int>((static_cast<int64_t>(blockIdx.x) * units) / gridDim.x);
+  u1 = static_cast<int>((static_cast<int64_t>(blockIdx.x + 1) * units) / gridDim.x);
+}
+
 __global__ void __launch_bounds__(kThreads, 1)
     quantize_act_kernel(const __grid_constant__ CUtensorMap tmap_x,
                         const __grid_constant__ CUtensorMap tmap_l1, const QuantParams p) {
@@ -81,20 +96,20 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t l1_bytes = static_cast<uint32_t>(p.r) * 128u;
   uint8_t* xs = base;
   uint8_t* ls = xs + kStages * kXTileBytes;
-  float* inv_s = reinterpret_cast<float*>(ls + kStages * l1_bytes);
-  uint64_t* full = reinterpret_cast<uint64_t*>(inv_s + p.kc);
+  float* inv_st = reinterpret_cast<float*>(ls + kStages * l1_bytes);  // [kStages][64]
+  uint64_t* full = reinterpret_cast<uint64_t*>(inv_st + kStages * kSubK);
   uint64_t* qdone = full + kStages;
   uint64_t* empty = qdone + kStages;
-  uint64_t* accf = empty + kStages;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accf + 1);
+  uint64_t* acc_full = empty + kStages;  // [2]
+  uint64_t* acc_empty = acc_full + 2;    // [2]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int m0 = blockIdx.x * kBM;
-  const int k_begin = blockIdx.y * p.kc;
-  const int k_end = min(p.K, k_begin + p.kc);
-  const int nsub = (k_end - k_begin) / kSubK;
+  const int kblocks = p.K / kSubK;
   const bool has_lr = p.r > 0;
-  const uint32_t tmem_cols = p.r <= 32 ? 32u : static_cast<uint32_t>(p.r);
+  const uint32_t tmem_cols = p.r <= 16 ? 32u : static_cast<uint32_t>(2 * p.r);
+  int u0, u1;
+  unit_range(p.units, u0, u1);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
@@ -102,15 +117,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&qdone[s], kQuantWarps);
       mbar_init(&empty[s], has_lr ? 1 : kQuantWarps);
     }
-    mbar_init(accf, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&acc_full[b], 1);
+      mbar_init(&acc_empty[b], kEpiWarps);
+    }
     fence_mbar_init();
   }
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tmap_x);
     if (has_lr) tma_prefetch_desc(&tmap_l1);
   }
-  for (int j = threadIdx.x; j < k_end - k_begin; j += kThreads)
-    inv_s[j] = p.smooth_s ? __fdiv_rn(1.0f, p.smooth_s[k_begin + j]) : 1.0f;
   if (warp == 1 && has_lr) {
     tmem_alloc(tmem_slot, tmem_cols);
     tmem_relinquish();
@@ -122,74 +138,92 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == 0) {
     // ------------------------------------------------------- producer ----
-    if (lane == 0) {
-      int issued = 0;
-      for (int i = 0; i < nsub; ++i) {
-        const int s = i % kStages;
-        const uint32_t ph = (i / kStages) & 1;
-        if (!mbar_wait(&empty[s], ph ^ 1, p.wait, kErrTimeoutEmpty)) break;
-        mbar_arrive_expect_tx(&full[s], kXTileBytes + (has_lr ? l1_bytes : 0u));
-        const int kc0 = k_begin + i * kSubK;
-        tma_load_2d(xs + s * kXTileBytes, &tmap_x, &full[s], kc0, m0);
-        if (has_lr) tma_load_2d(ls + s * l1_bytes, &tmap_l1, &full[s], kc0, 0);
-        issued = i + 1;
+    int issued = 0;
+    for (int u = u0; u < u1; ++u) {
+      const int i = u - u0;
+      const int s = i % kStages;
+      const uint32_t ph = (i / kStages) & 1;
+      int ok = 1;
+      if (lane == 0) ok = mbar_wait(&empty[s], ph ^ 1, p.wait, kErrTimeoutEmpty) ? 1 : 0;
+      if (!__shfl_sync(0xffffffffu, ok, 0)) break;
+      const int rb = u / kblocks, kb = u % kblocks;
+      // RN(1/s) of this slot's 64 columns, published by the arrive below
+      float2 iv = make_float2(1.0f, 1.0f);
+      if (p.smooth_s) {
+        const float2 sv = *reinterpret_cast<const float2*>(p.smooth_s + kb * kSubK + 2 * lane);
+        iv = make_float2(__fdiv_rn(1.0f, sv.x), __fdiv_rn(1.0f, sv.y));
       }
-      // never leave the CTA with a copy still landing in its shared memory
+      reinterpret_cast<float2*>(inv_st + s * kSubK)[lane] = iv;
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive_expect_tx(&full[s], kXTileBytes + (has_lr ? l1_bytes : 0u));
+        tma_load_2d(xs + s * kXTileBytes, &tmap_x, &full[s], kb * kSubK, rb * kBM);
+        if (has_lr) tma_load_2d(ls + s * l1_bytes, &tmap_l1, &full[s], kb * kSubK, 0);
+      }
+      issued = i + 1;
+    }
+    // never leave the CTA with a copy still landing in its shared memory
+    if (lane == 0)
       for (int i = max(0, issued - kStages); i < issued; ++i)
         mbar_wait(&full[i % kStages], (i / kStages) & 1, p.wait, kErrTimeoutDrain);
-    }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA ----
     if (has_lr && lane == 0) {
       const uint32_t idesc = idesc_f16(128, static_cast<uint32_t>(p.r), true);
-      bool ok = true;
-      for (int i = 0; i < nsub; ++i) {
+      int seg = 0;             // segments started by this CTA
+      bool first = true;       // first sub-tile of the current segment
+      for (int u = u0; u < u1; ++u) {
+        const int i = u - u0;
         const int s = i % kStages;
         const uint32_t ph = (i / kStages) & 1;
-        if (!mbar_wait(&qdone[s], ph, p.wait, kErrTimeoutFull)) {
-          ok = false;
+        const int buf = seg & 1;
+        if (first && seg >= 2 &&
+            !mbar_wait(&acc_empty[buf], ((seg >> 1) - 1) & 1, p.wait, kErrTimeoutAcc))
           break;
-        }
+        if (!mbar_wait(&qdone[s], ph, p.wait, kErrTimeoutFull)) break;
         tc_fence_after();
         const uint32_t a0 = smem_u32(xs + s * kXTileBytes);
         const uint32_t b0 = smem_u32(ls + s * l1_bytes);
+        const uint32_t d = tmem + buf * static_cast<uint32_t>(p.r);
 #pragma unroll
         for (int kk = 0; kk < kSubK / 16; ++kk) {
           const uint64_t ad = make_sdesc(a0 + kk * 32, 16, 1024, kSwz128);
           const uint64_t bd = make_sdesc(b0 + kk * 32, 16, 1024, kSwz128);
-          umma_f16(tmem, ad, bd, idesc, (i > 0 || kk > 0) ? 1u : 0u);
+          umma_f16(d, ad, bd, idesc, (!first || kk > 0) ? 1u : 0u);
         }
         umma_commit(&empty[s]);
+        first = false;
+        const bool seg_end = (u + 1 == u1) || ((u + 1) / kblocks != u / kblocks);
+        if (seg_end) {
+          umma_commit(&acc_full[buf]);
+          ++seg;
+          first = true;
+        }
       }
-      if (ok) umma_commit(accf);
     }
-  } else {
+  } else if (warp < 2 + kQuantWarps) {
     // ------------------------------------------------------ quantizers ----
     const int qw = warp - 2;
     const int row = 32 * (qw & 3) + lane;  // row within the tile
     const int half = qw >> 2;              // which 32 of the 64 columns
-    const int grow = m0 + row;
     float gs;
     if (p.gs_in) {
       gs = *p.gs_in;
     } else {
       gs = tensor_scale_from_amax(*p.amax_src);
     }
-    if (p.gs_copy && blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 64) *p.gs_copy = gs;
+    if (p.gs_copy && blockIdx.x == 0 && threadIdx.x == 64) *p.gs_copy = gs;
     const size_t kbytes = static_cast<size_t>(p.K) / 2;
-    const int kblocks = p.K / 64;
-    uint8_t* sf_row = p.sf_out + static_cast<size_t>(m0 / 128) * kblocks * 512 + (row & 31) * 16 +
-                      (row >> 5) * 4 + 2 * half;
-    bool ok = true;
-    for (int i = 0; i < nsub; ++i) {
+    for (int u = u0; u < u1; ++u) {
+      const int i = u - u0;
       const int s = i % kStages;
       const uint32_t ph = (i / kStages) & 1;
-      if (!mbar_wait(&full[s], ph, p.wait, kErrTimeoutFull)) {
-        ok = false;
-        break;
-      }
+      if (!mbar_wait(&full[s], ph, p.wait, kErrTimeoutFull)) break;
+      const int rb = u / kblocks, kb = u % kblocks;
+      const int grow = rb * kBM + row;
       uint8_t* trow = xs + s * kXTileBytes + row * 128;
-      const int kt = i * kSubK + 32 * half;  // column offset within this CTA's range
+      const int kc0 = kb * kSubK + 32 * half;  // first column of this thread
+      const float* inv_s = inv_st + s * kSubK + 32 * half;
       uint4 v[4];
 #pragma unroll
       for (int j = 0; j < 4; ++j)
@@ -202,7 +236,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t w[8] = {v[2 * g].x,     v[2 * g].y,     v[2 * g].z,     v[2 * g].w,
                                v[2 * g + 1].x, v[2 * g + 1].y, v[2 * g + 1].z, v[2 * g + 1].w};
         float xh[16];
-        const float4* is4 = reinterpret_cast<const float4*>(inv_s + kt + 16 * g);
+        const float4* is4 = reinterpret_cast<const float4*>(inv_s + 16 * g);
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
           const float4 iv = is4[q];
@@ -238,15 +272,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                                          pack_bf16x2(xh[8 * h + 6], xh[8 * h + 7]));
         }
       }
-      const int kc0 = k_begin + i * kSubK;
       if (grow < p.M) {
-        *reinterpret_cast<uint4*>(p.q_out + static_cast<size_t>(grow) * kbytes +
-                                  (kc0 + 32 * half) / 2) =
+        *reinterpret_cast<uint4*>(p.q_out + static_cast<size_t>(grow) * kbytes + kc0 / 2) =
             make_uint4(codes[0], codes[1], codes[2], codes[3]);
       }
       // rows past M inside the last 128-row block hold zero-filled x, so
       // their scales are written as the zero padding the layout requires
-      *reinterpret_cast<uint16_t*>(sf_row + static_cast<size_t>(kc0 / 64) * 512) =
+      *reinterpret_cast<uint16_t*>(p.sf_out + (static_cast<size_t>(rb) * kblocks + kb) * 512 +
+                                   (row & 31) * 16 + (row >> 5) * 4 + 2 * half) =
           static_cast<uint16_t>(sfb[0] | (sfb[1] << 8));
       if (has_lr) {
 #pragma unroll
@@ -260,20 +293,25 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) mbar_arrive(&empty[s]);
       }
     }
-    // ------------------------------------------- down-projection out ----
-    if (has_lr && ok) {
-      if (mbar_wait(accf, 0, p.wait, kErrTimeoutAcc)) {
+  } else {
+    // ------------------------------------------------- xl epilogue ----
+    if (has_lr) {
+      const int quad = warp & 3;
+      int seg = 0;
+      for (int u = u0; u < u1; ++u) {
+        const bool seg_end = (u + 1 == u1) || ((u + 1) / kblocks != u / kblocks);
+        if (!seg_end) continue;
+        const int buf = seg & 1;
+        if (!mbar_wait(&acc_full[buf], (seg >> 1) & 1, p.wait, kErrTimeoutAcc)) break;
         tc_fence_after();
-        const int quad = warp & 3;
-        const int set = qw >> 2;
-        const int grow_acc = m0 + 32 * quad + lane;
-        for (int c = set; c < p.r / 16; c += 2) {
+        const int grow = (u / kblocks) * kBM + 32 * quad + lane;
+        const uint32_t taddr = tmem + (static_cast<uint32_t>(32 * quad) << 16) + buf * p.r;
+        for (int c = 0; c < p.r / 16; ++c) {
           uint32_t acc[16];
-          tmem_ld_32x32b_x16(tmem + (static_cast<uint32_t>(32 * quad) << 16) + c * 16, acc);
+          tmem_ld_32x32b_x16(taddr + c * 16, acc);
           tmem_ld_wait();
-          if (grow_acc < p.M) {
-            float4* dst = reinterpret_cast<float4*>(p.lora_out + static_cast<size_t>(grow_acc) * p.r +
-                                                    c * 16);
+          if (grow < p.M) {
+            float4* dst = reinterpret_cast<float4*>(p.lora_out + static_cast<size_t>(grow) * p.r + c * 16);
 #pragma unroll
             for (int q = 0; q < 4; ++q)
               atomicAdd(dst + q, make_float4(__uint_as_float(acc[4 * q]), __uint_as_float(acc[4 * q + 1]),
@@ -281,6 +319,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                                              __uint_as_float(acc[4 * q + 3])));
           }
         }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&acc_empty[buf]);
+        ++seg;
       }
     }
   }
@@ -336,6 +378,8 @@ svdq_status launch_quantize_act(const LaunchCtx& ctx, const void* x, int64_t M, 
                                 int64_t ldx, const float* smooth_s, const void* L1t, int r,
                                 const float* act_gscale, float* act_gscale_out, uint8_t* q_out,
                                 uint8_t* sf_out, float* lora_out) {
+  if (smooth_s && (reinterpret_cast<uintptr_t>(smooth_s) & 7))
+    return fail(SVDQ_ERR_MISALIGNED, "smooth_s must be 8-byte aligned");
   CUtensorMap tx{}, tl{};
   if (!make_tmap_2d(&tx, x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, M, K, ldx * 2, kBM, kSubK, 128))
     return SVDQ_ERR_CUDA;
@@ -344,21 +388,11 @@ svdq_status launch_quantize_act(const LaunchCtx& ctx, const void* x, int64_t M, 
     return SVDQ_ERR_CUDA;
   if (r == 0) tl = tx;
 
-  const int gx = static_cast<int>((M + kBM - 1) / kBM);
-  int kc = 64;
-  for (int c : {1024, 512, 256, 128}) {
-    if (static_cast<int64_t>(gx) * ((K + c - 1) / c) >= 2 * ctx.num_sms) {
-      kc = c;
-      break;
-    }
-  }
-  const int gy = static_cast<int>((K + kc - 1) / kc);
-
   QuantParams p{};
   p.M = static_cast<int>(M);
   p.K = static_cast<int>(K);
   p.r = r;
-  p.kc = kc;
+  p.units = static_cast<int>(((M + kBM - 1) / kBM) * (K / kSubK));
   p.smooth_s = smooth_s;
   p.gs_in = act_gscale;
   p.amax_src = act_gscale ? nullptr : act_gscale_out;
@@ -380,15 +414,16 @@ svdq_status launch_quantize_act(const LaunchCtx& ctx, const void* x, int64_t M, 
                                                   smooth_s, reinterpret_cast<unsigned*>(act_gscale_out));
     if (svdq_status e = check_launch("act_amax_kernel")) return e;
   }
-  const size_t smem = 1024 + kStages * (kXTileBytes + static_cast<size_t>(r) * 128) +
-                      static_cast<size_t>(kc) * 4 + 8 * (3 * kStages + 1) + 16;
+  const size_t smem = 1024 + kStages * (kXTileBytes + static_cast<size_t>(r) * 128 + kSubK * 4) +
+                      8 * (3 * kStages + 4) + 16;
   static bool attr_done[64] = {};
   if (!attr_done[ctx.device & 63]) {
     cudaFuncSetAttribute(quantize_act_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          227 * 1024);
     attr_done[ctx.device & 63] = true;
   }
-  quantize_act_kernel<<<dim3(gx, gy), kThreads, smem, st>>>(tx, tl, p);
+  const int grid = std::min(p.units, ctx.num_sms);
+  quantize_act_kernel<<<grid, kThreads, smem, st>>>(tx, tl, p);
   if (svdq_status e = check_launch("quantize_act_kernel")) return e;
   if (!act_gscale) {
     act_scale_finalize_kernel<<<1, 1, 0, st>>>(act_gscale_out);

@@ -77,6 +77,8 @@ def test_linear_and_awq_validation_is_host_side():
     st = L.awq_w4a16_linear(v(16), 8, 8192, None, v(16), v(16), v(16), 64, None, 32, v(16), None)
     assert st == sv.INVALID_ARG  # K too large for the B table at M > 4
     assert b"K=8192" in L.svdq_last_error_detail()
+    st = L.awq_w4a16_linear(v(16), 4, 14464, None, v(16), v(16), v(16), 64, None, 32, v(16), None)
+    assert st == sv.INVALID_ARG  # K over the M <= 4 limit
 
 
 def test_unsupported_device_is_a_clear_error(monkeypatch):
