@@ -100,7 +100,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* full = reinterpret_cast<uint64_t*>(base + L::kRing + L::kBias);
   uint64_t* empty = full + kStages;
   uint64_t* lrf = empty + kStages;       // low-rank A written, per ring slot
-  uint64_t* acc_full = lrf + kStages;
+  // Slot free for a low-rank A write.  The epilogue cannot wait on empty[s]
+  // for that: it looks several ring steps ahead, and a parity wait cannot
+  // tell phase p from p + 2.  lrfree[s] completes one phase per low-rank use
+  // of slot s (committed by the MMA when the slot's previous step is done),
+  // so it can never run more than one phase ahead of the epilogue.
+  uint64_t* lrfree = lrf + kStages;
+  uint64_t* acc_full = lrfree + kStages;
   uint64_t* acc_empty = acc_full + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 1);
   auto stage_a = [&](int s) { return base + s * L::kStage; };
@@ -121,6 +127,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
       mbar_init(&lrf[s], kEpiWarps / 2);
+      mbar_init(&lrfree[s], 1);
     }
     mbar_init(acc_full, 1);
     mbar_init(acc_empty, kEpiWarps);
@@ -249,6 +256,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           }
           umma_commit(&empty[s]);
+          // the step kStages ahead reuses this slot; if it is a low-rank step,
+          // tell the epilogue when this step's reads of the slot are done
+          if ((it + kStages) % nsteps >= nk) umma_commit(&lrfree[s]);
         }
         if (ok) umma_commit(acc_full);
       }
@@ -263,6 +273,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const float alpha = __fdiv_rn(1.0f, gprod);
     constexpr int kCols = L::kColsPerWarp;
     int it = 0;
+    uint32_t free_par = 0;                   // parity of each slot's next lrfree phase
     int local = 0;
     bool ok = true;
     for (int t = blockIdx.x; ok && t < p.tiles; t += gridDim.x, ++local) {
@@ -285,10 +296,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int j = 0; j < nlr; ++j, ++it) {
         const int s = it % kStages;
         const uint32_t ph = (it / kStages) & 1;
+        (void)ph;
         if (half != 0) continue;
-        if (!mbar_wait(&empty[s], ph ^ 1, p.wait, kErrTimeoutEmpty)) {
-          ok = false;
-          break;
+        if (it >= kStages) {  // the slot had a previous user: wait until it is done
+          if (!mbar_wait(&lrfree[s], (free_par >> s) & 1u, p.wait, kErrTimeoutEmpty)) {
+            ok = false;
+            break;
+          }
+          free_par ^= 1u << s;
         }
         uint8_t* arow = stage_a(s) + row * 128;
 #pragma unroll
@@ -378,7 +393,7 @@ template <int BN>
 svdq_status launch_bn(const LaunchCtx& ctx, const CUtensorMap& ta, const CUtensorMap& tb,
                       const CUtensorMap& tl, GemmParams p) {
   using L = Layout<BN>;
-  const size_t smem = 1024 + static_cast<size_t>(L::kRing) + L::kBias + 8 * (3 * kStages + 2) + 16;
+  const size_t smem = 1024 + static_cast<size_t>(L::kRing) + L::kBias + 8 * (4 * kStages + 2) + 16;
   static bool attr_done[64] = {};
   if (!attr_done[ctx.device & 63]) {
     cudaFuncSetAttribute(w4a4_gemm_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,

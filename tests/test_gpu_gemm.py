@@ -156,3 +156,34 @@ def test_fused_qkv_rank_sweep_full_size(r):
     d, L = _full(workloads.QKV[r].name, r)
     y, ref = _whole_layer_sampled(d, L, step=32)
     assert_gemm_close(y, ref, f"qkv r={r}")
+
+
+def _random_operands(M, K, N, r, seed):
+    """Oracle-quantized random operands (no SVD) for shapes with many tiles."""
+    from oracle import codecs
+    rng = np.random.default_rng(seed)
+    x = workloads.to_bf16(rng.standard_normal((M, K)).astype(np.float32))
+    q = osv.quantize_act(x, None)
+    R = rng.standard_normal((N, K)).astype(np.float32) * 0.05
+    gs_w = osv.tensor_scale(np.abs(R).max())
+    cw, sfw = osv.nvfp4_quantize(R, gs_w)
+    L1t = workloads.to_bf16(rng.standard_normal((r, K)).astype(np.float32) * 0.05)
+    L2t = workloads.to_bf16(rng.standard_normal((N, r)).astype(np.float32) * 0.2)
+    bias = workloads.to_bf16(rng.standard_normal(N).astype(np.float32) * 0.01)
+    xl = osv.lora_down(x, None, L1t)
+    L = dict(packed_w=codecs.pack_nibbles(cw), sf_w_swizzled=codecs.swizzle_scales(sfw), gs_w=gs_w,
+             L1t=L1t, L2t=L2t, s=None, bias=bias)
+    return q, xl, cw, sfw, gs_w, L
+
+
+@pytest.mark.parametrize("M,K,N,r", [(512, 1536, 20480, 32), (256, 3072, 10240, 64), (384, 2048, 9984, 128)])
+def test_gemm_many_tiles_per_cta(M, K, N, r):
+    # more output tiles than SMs, and more K steps than ring slots: every CTA
+    # walks several tiles and the ring wraps inside each tile
+    q, xl, cw, sfw, gs_w, L = _random_operands(M, K, N, r, seed=M + N)
+    y = sv.w4a4_linear(u8(q["packed"]), u8(q["sf_swizzled"]), f32([q["gs"]]), f32(xl), weights_from_layer(L))
+    torch.cuda.synchronize()
+    cols = np.sort(np.random.default_rng(0).choice(N, 768, replace=False))
+    ref = osv.svdq_linear(q["codes"], q["sf"], q["gs"], xl, cw[cols], sfw[cols], gs_w, L["L2t"][cols],
+                          L["bias"][cols])
+    assert_gemm_close(y[:, torch.from_numpy(cols).cuda()], ref, f"many tiles M{M} K{K} N{N} r{r}")

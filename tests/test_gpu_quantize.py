@@ -130,3 +130,22 @@ def test_signed_zero_and_saturation_codes():
         ref = osv.quantize_act(x, None, gs)
         assert np.array_equal(sf, ref["sf_swizzled"]), describe_byte_mismatch(sf, ref["sf_swizzled"])
         assert np.array_equal(q, ref["packed"]), describe_byte_mismatch(q.ravel(), ref["packed"].ravel())
+
+
+@pytest.mark.parametrize("M,K,r", [(1024, 4096, 32), (640, 3072, 128), (1000, 2048, 0)])
+def test_quantize_many_units_per_cta(M, K, r):
+    # more 128x64 sub-tiles than SMs: every CTA walks a range that crosses
+    # row blocks, so the down-projection accumulators alternate
+    rng = np.random.default_rng(M + K + r)
+    x = workloads.to_bf16(rng.standard_normal((M, K)).astype(np.float32))
+    s = rng.uniform(0.5, 2.0, K).astype(np.float32)
+    L1t = workloads.to_bf16(rng.standard_normal((max(r, 16), K)).astype(np.float32) * 0.05)[:r]
+    L = dict(s=s, L1t=L1t)
+    gs_ref = osv.act_tensor_scale(x, s)
+    q, sf, lora, gs = _run(x, L, r, False, gs_ref)
+    ref = osv.quantize_act(x, s, gs_ref)
+    assert np.array_equal(sf, ref["sf_swizzled"]), describe_byte_mismatch(sf, ref["sf_swizzled"])
+    assert np.array_equal(q, ref["packed"]), describe_byte_mismatch(q.ravel(), ref["packed"].ravel())
+    if r:
+        xl_ref = osv.lora_down(x, s, L1t)
+        assert np.linalg.norm(lora - xl_ref) <= 1e-4 * np.linalg.norm(xl_ref)
