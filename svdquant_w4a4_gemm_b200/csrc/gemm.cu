@@ -10,28 +10,41 @@
 // its activation operand keeps ~16 significant bits through the hi/lo
 // split; L2 itself is bf16 by construction.
 //
-// Persistent kernel: one CTA per SM walks 128 x BN output tiles (BN = 256,
-// or 128 when N is not a multiple of 256); fp32 accumulator in TMEM.
-//   warp 0     producer.  For each tile: the FP4 steps (TMA of 128-byte rows
-//              of packed A and B = 256 K-elements, 128-byte swizzle; bulk
-//              copies of the matching scale blocks — the 128x4 block layout
-//              is already the byte order the scale copy to TMEM wants),
-//              then the low-rank steps (TMA of a 64-wide slice of L2ᵀ).
-//              All go through one kStages-deep shared-memory ring.
-//   warp 1     TMEM owner and MMA issuer (one thread).  Per FP4 step:
-//              tcgen05.cp of the scale blocks into TMEM (4 columns per 128
-//              rows per 64 K), four block-scaled MMAs (K = 64 each).  Per
-//              low-rank step: kind::f16 MMAs into the same accumulator.
-//              tcgen05.commit frees ring slots and, after a tile's last
-//              step, hands the accumulator to the epilogue.
-//   warps 2-9  epilogue, two warps per 32-lane TMEM quadrant (one per half
-//              of BN).  During a tile's mainloop they write the tile's
-//              low-rank A operand (hi/lo bf16 of the fp32 down-projection,
-//              swizzled by hand) into the ring slots of its low-rank steps
-//              and stage the bias slice in shared memory; after the
-//              accumulator is full they drain TMEM -> registers (α·acc +
-//              bias -> bf16), release the accumulator to the MMA warp and
-//              store y while the next tile's mainloop runs.
+// Persistent kernel: one CTA per SM walks 128 x BN output tiles (BN = 192
+// when N is a multiple of 192, else 128).  Tensor memory holds two fp32
+// accumulators (the epilogue drains one while the MMAs fill the other) and
+// two scale-factor regions (the stagers fill one while the MMAs read the
+// other): 2·BN + 2·48 <= 512 columns.
+//   warp 0      producer: per FP4 step (256 K) bulk copies of the matching
+//               128x4 scale blocks (first, on their own barrier, so that the
+//               stagers can start while the operands land), then TMA of
+//               packed A (128 rows x 128 B) and B (BN rows x 128 B) with
+//               128-byte swizzle; per low-rank step (32 of the r columns)
+//               TMA of the L2ᵀ slice and of the tile's fp32 xl slice (into
+//               the A slot).  One kStages-deep ring.
+//   warp 1      TMEM owner and MMA issuer (one thread): four block-scaled
+//               MMAs (K = 64 each) per FP4 step, then the low-rank kind::f16
+//               MMAs, into the tile's accumulator; tcgen05.commit frees ring
+//               slots and scale regions and, at the end of a tile, hands the
+//               accumulator to the epilogue.
+//   warps 2-5   stagers, one per 32-lane TMEM quadrant.  Per FP4 step they
+//               move the step's E4M3 scales from shared memory into a scale
+//               region with tcgen05.st, every quadrant holding the same
+//               copy (lane l, column j: the 4 scales of row 32j + l per
+//               64-K block, the order the block-scaled MMA reads).  Stores
+//               from registers run beside the MMAs; a shared-to-TMEM copy
+//               issued by the MMA thread would queue behind them.  Per
+//               low-rank step they turn the slot's xl slice in place into
+//               the low-rank A operand: 32 columns of hi and 32 of lo (bf16
+//               of xl·gs_a·gs_w and of its remainder), swizzled by hand.
+//               The MMA thread waits on one barrier per step (the stagers'),
+//               and keeps nothing but MMA issue on its path: the tensor pipe
+//               holds only about one MMA ahead, so any latency in the issuing
+//               thread shows up as idle tensor cycles.
+//   warps 6-13  epilogue, two per quadrant: TMEM -> registers (α·acc + bias
+//               -> bf16), release the accumulator, then 32 x 64 staging
+//               boxes in shared memory and TMA stores of y (full-line
+//               writes, clipped at the M and N edges).
 #include "internal.h"
 #include "ptx.cuh"
 
@@ -41,9 +54,11 @@ namespace {
 constexpr int kBM = 128;
 constexpr int kBKBytes = 128;  // 256 FP4 elements per FP4 step and row
 constexpr int kStages = 4;
+constexpr int kStagerWarps = 4;
 constexpr int kEpiWarps = 8;
-constexpr int kThreads = 32 * (2 + kEpiWarps);
+constexpr int kThreads = 32 * (2 + kStagerWarps + kEpiWarps);
 constexpr uint32_t kATileBytes = kBM * kBKBytes;  // 16 KB
+constexpr uint32_t kSfRegionCols = 48;            // SFA 4 x 4 + SFB 4 x 8 columns
 
 struct GemmParams {
   int M, N, K, r;
@@ -52,10 +67,7 @@ struct GemmParams {
   const uint8_t* sf_w;
   const float* gs_a;
   const float* gs_w;
-  const float* lora;      // [M, r]
   const uint16_t* bias;   // [N] or null
-  uint16_t* y;
-  int64_t ldy;
   int fault;              // test hook: 1 = the first ring slot never fills
   WaitCfg wait;
 };
@@ -69,16 +81,17 @@ template <int BN>
 struct Layout {
   static constexpr uint32_t kB = BN * kBKBytes;          // B tile bytes
   static constexpr uint32_t kSfa = 4 * 512;              // 4 K-blocks x 128 rows
-  static constexpr uint32_t kSfb = (BN / 128) * 4 * 512;
+  static constexpr uint32_t kSfb = 2 * 4 * 512;          // up to two 128-row blocks
   static constexpr uint32_t kStage = kATileBytes + kB + kSfa + kSfb;
   static constexpr uint32_t kRing = kStages * kStage;
-  static constexpr uint32_t kBias = kEpiWarps * (BN / 2) * 2;  // per-warp bias slices
-  static constexpr uint32_t kTmemCols = BN == 256 ? 512 : 256;
-  static constexpr uint32_t kSfaCol = BN;                // 16 columns
-  static constexpr uint32_t kSfbCol = BN + 16;           // (BN/128)*16 columns
-  static constexpr int kColsPerWarp = BN / 2;            // epilogue columns per warp
+  static constexpr int kBoxes = BN / 64;                 // 64-column store boxes per tile
+  static constexpr int kBoxes0 = (kBoxes + 1) / 2;       // boxes of the half-0 epilogue warps
+  static constexpr uint32_t kBoxBytes = 32 * 128;        // 32 rows x 64 bf16
+  static constexpr uint32_t kBias = kEpiWarps * kBoxes0 * 64 * 2;
+  static constexpr uint32_t kSfCol = 2 * BN;             // first scale-region column
   static_assert(kStage % 1024 == 0, "stage must keep 1 KB alignment");
-  static_assert(BN + 16 + (BN / 128) * 16 <= kTmemCols, "TMEM budget");
+  static_assert(2 * BN + 2 * kSfRegionCols <= 512, "TMEM budget");
+  static_assert(BN % 64 == 0 && BN <= 256, "tile width");
 };
 
 // Where tile `t` sits in the output.
@@ -91,55 +104,61 @@ template <int BN>
 __global__ void __launch_bounds__(kThreads, 1)
     w4a4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
                      const __grid_constant__ CUtensorMap tmap_b,
-                     const __grid_constant__ CUtensorMap tmap_l2, const GemmParams p) {
+                     const __grid_constant__ CUtensorMap tmap_l2,
+                     const __grid_constant__ CUtensorMap tmap_y,
+                     const __grid_constant__ CUtensorMap tmap_lr, const GemmParams p) {
   using L = Layout<BN>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
-  uint16_t* bias_s = reinterpret_cast<uint16_t*>(base + L::kRing);
-  uint64_t* full = reinterpret_cast<uint64_t*>(base + L::kRing + L::kBias);
-  uint64_t* empty = full + kStages;
+  uint8_t* out_s = base + L::kRing;                                     // [kEpiWarps][box]
+  uint16_t* bias_s = reinterpret_cast<uint16_t*>(out_s + kEpiWarps * L::kBoxBytes);
+  uint64_t* full = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(bias_s) + L::kBias);
+  uint64_t* full_sf = full + kStages;    // the slot's scale blocks landed (FP4 steps only)
+  uint64_t* empty = full_sf + kStages;
   uint64_t* lrf = empty + kStages;       // low-rank A written, per ring slot
-  // Slot free for a low-rank A write.  The epilogue cannot wait on empty[s]
-  // for that: it looks several ring steps ahead, and a parity wait cannot
-  // tell phase p from p + 2.  lrfree[s] completes one phase per low-rank use
-  // of slot s (committed by the MMA when the slot's previous step is done),
-  // so it can never run more than one phase ahead of the epilogue.
-  uint64_t* lrfree = lrf + kStages;
-  uint64_t* acc_full = lrfree + kStages;
-  uint64_t* acc_empty = acc_full + 1;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 1);
+  uint64_t* sfready = lrf + kStages;     // [2] scale region written (and the slot's operands landed)
+  uint64_t* sffree = sfready + 2;        // [2] scale region read by its MMAs
+  uint64_t* acc_full = sffree + 2;       // [2]
+  uint64_t* acc_empty = acc_full + 2;    // [2]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
   auto stage_a = [&](int s) { return base + s * L::kStage; };
   auto stage_b = [&](int s) { return base + s * L::kStage + kATileBytes; };
   auto stage_sfa = [&](int s) { return base + s * L::kStage + kATileBytes + L::kB; };
   auto stage_sfb = [&](int s) { return base + s * L::kStage + kATileBytes + L::kB + L::kSfa; };
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const bool lr_packed = p.r > 0 && p.r <= 32;  // hi and lo share one A tile
-  const int nlr = p.r == 0 ? 0 : (lr_packed ? 1 : 2 * (p.r / 64));  // low-rank steps per tile
+  // low-rank steps per tile: 32 columns of r each (r = 16: one, zero-padded)
+  const int nlr = p.r == 0 ? 0 : (p.r <= 32 ? 1 : p.r / 32);
   const int kblocks = p.K / 64;              // 64-element K blocks (one MMA each)
-  const int nk = (kblocks + 3) / 4;          // FP4 steps per tile (last may be short)
+  const int nk = (kblocks + 3) / 4;          // FP4 steps per tile (the last may be short)
   const int nsteps = nk + nlr;               // ring steps per tile
   const int nb_total = (p.N + 127) / 128;    // 128-row blocks of the weight scales
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&full[s], 1);
+      mbar_init(&full_sf[s], 1);
       mbar_init(&empty[s], 1);
-      mbar_init(&lrf[s], kEpiWarps / 2);
-      mbar_init(&lrfree[s], 1);
+      mbar_init(&lrf[s], kStagerWarps);
     }
-    mbar_init(acc_full, 1);
-    mbar_init(acc_empty, kEpiWarps);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&sfready[b], kStagerWarps);
+      mbar_init(&sffree[b], 1);
+      mbar_init(&acc_full[b], 1);
+      mbar_init(&acc_empty[b], kEpiWarps);
+    }
     fence_mbar_init();
   }
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tmap_a);
     tma_prefetch_desc(&tmap_b);
     if (p.r > 0) tma_prefetch_desc(&tmap_l2);
+    if (p.r > 0) tma_prefetch_desc(&tmap_lr);
+    tma_prefetch_desc(&tmap_y);
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, L::kTmemCols);
+    tmem_alloc(tmem_slot, 512);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -150,13 +169,17 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0) {
     // ------------------------------------------------------- producer ----
     if (lane == 0) {
-      int it = 0;          // ring step counter (continues across tiles)
-      int issued_to = 0;   // ring steps whose loads were issued
+      int it = 0;              // ring step counter (continues across tiles)
+      uint32_t used = 0;       // slots that received loads
+      uint32_t sf_used = 0;    // slots that received scale blocks
+      uint32_t full_par = 0;   // per slot: parity of its next full phase
+      uint32_t sf_par = 0;     // per slot: parity of its next full_sf phase
       bool ok = true;
       for (int t = blockIdx.x; ok && t < p.tiles; t += gridDim.x) {
         int m0, n0;
         tile_coords(t, p.tiles_n, BN, m0, n0);
-        const int nbl = min(BN / 128, nb_total - n0 / 128);  // weight scale row blocks
+        const int b0 = n0 / 128;  // first weight-scale block of the tile
+        const int nbl = min((n0 + BN - 1) / 128, nb_total - 1) - b0 + 1;
         for (int st = 0; st < nsteps; ++st, ++it) {
           const int s = it % kStages;
           const uint32_t ph = (it / kStages) & 1;
@@ -166,32 +189,40 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           if (st < nk) {
             if (p.fault == 1 && it == 0) continue;  // test hook: this slot never fills
-            const int kb = st;                      // 256-element K step
-            const int nkb = min(4, kblocks - 4 * kb);
+            const int nkb = min(4, kblocks - 4 * st);
             const uint32_t sfbytes = static_cast<uint32_t>(nkb) * 512;
-            mbar_arrive_expect_tx(&full[s], kATileBytes + L::kB + sfbytes * (1 + nbl));
-            tma_load_2d(stage_a(s), &tmap_a, &full[s], kb * kBKBytes, m0);
-            tma_load_2d(stage_b(s), &tmap_b, &full[s], kb * kBKBytes, n0);
-            bulk_load(stage_sfa(s), p.sf_a + (static_cast<size_t>(m0 / 128) * kblocks + 4 * kb) * 512,
-                      sfbytes, &full[s]);
+            mbar_arrive_expect_tx(&full_sf[s], sfbytes * (1 + nbl));
+            bulk_load(stage_sfa(s), p.sf_a + (static_cast<size_t>(m0 / 128) * kblocks + 4 * st) * 512,
+                      sfbytes, &full_sf[s]);
             for (int nb = 0; nb < nbl; ++nb)
               bulk_load(stage_sfb(s) + nb * 2048,
-                        p.sf_w + (static_cast<size_t>(n0 / 128 + nb) * kblocks + 4 * kb) * 512,
-                        sfbytes, &full[s]);
+                        p.sf_w + (static_cast<size_t>(b0 + nb) * kblocks + 4 * st) * 512, sfbytes,
+                        &full_sf[s]);
+            sf_used |= 1u << s;
+            sf_par ^= 1u << s;
+            mbar_arrive_expect_tx(&full[s], kATileBytes + L::kB);
+            tma_load_2d(stage_a(s), &tmap_a, &full[s], st * kBKBytes, m0);
+            tma_load_2d(stage_b(s), &tmap_b, &full[s], st * kBKBytes, n0);
           } else {
-            // L2ᵀ[n0 .. n0+BN) x r[64c .. 64c+64) as bf16, zero-filled past r
+            // L2ᵀ[n0 .. n0+BN) x r[32j .. 32j+64) as bf16 (only the first 32
+            // columns are used) and xl[m0 .. m0+128) x r[32j .. 32j+32) as
+            // fp32; both zero-filled past M, N and r
             const int j = st - nk;
-            const int c = lr_packed ? 0 : j / 2;
-            mbar_arrive_expect_tx(&full[s], L::kB);
-            tma_load_2d(stage_b(s), &tmap_l2, &full[s], 64 * c, n0);
+            mbar_arrive_expect_tx(&full[s], L::kB + kATileBytes);
+            tma_load_2d(stage_b(s), &tmap_l2, &full[s], 32 * j, n0);
+            tma_load_2d(stage_a(s), &tmap_lr, &full[s], 32 * j, m0);
           }
-          issued_to = it + 1;
+          used |= 1u << s;
+          full_par ^= 1u << s;
         }
       }
-      // never leave the CTA with a copy still landing in its shared memory
-      for (int i = max(0, issued_to - kStages); i < issued_to; ++i) {
-        if (p.fault == 1 && i == 0) continue;
-        mbar_wait(&full[i % kStages], (i / kStages) & 1, p.wait, kErrTimeoutDrain);
+      // never leave the CTA with a copy still landing in its shared memory:
+      // every earlier phase of a slot completed before the slot was reused
+      for (int s = 0; s < kStages; ++s) {
+        if (used & (1u << s))
+          mbar_wait(&full[s], ((full_par >> s) & 1u) ^ 1u, p.wait, kErrTimeoutDrain);
+        if (sf_used & (1u << s))
+          mbar_wait(&full_sf[s], ((sf_par >> s) & 1u) ^ 1u, p.wait, kErrTimeoutDrain);
       }
     }
   } else if (warp == 1) {
@@ -199,45 +230,43 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       const uint32_t id_f16 = idesc_f16(128, BN, true);
       const uint32_t id_fp4 = idesc_nvfp4(128, BN);
-      int it = 0;
-      uint32_t lr_par = 0;                   // parity of each slot's next low-rank phase
+      // descriptors of slot 0, k-offset 0; a slot / k offset adds (bytes >> 4)
+      // to the start-address field (shared addresses stay below 256 KB)
+      const uint64_t da0 = make_sdesc(smem_u32(stage_a(0)), 16, 1024, kSwz128);
+      const uint64_t db0 = make_sdesc(smem_u32(stage_b(0)), 16, 1024, kSwz128);
+      int it = 0, f = 0;                     // ring steps, FP4 steps
+      uint32_t lr_par = 0;                   // parity of each slot's next lrf phase
       int local = 0;                         // tiles done by this CTA
       bool ok = true;
       for (int t = blockIdx.x; ok && t < p.tiles; t += gridDim.x, ++local) {
-        // the epilogue must have drained the previous tile's accumulator
-        if (local > 0 && !mbar_wait(acc_empty, (local - 1) & 1, p.wait, kErrTimeoutAcc)) {
+        const int a = local & 1;
+        const uint32_t acc = tmem + a * BN;
+        // the epilogue must have drained this accumulator's previous tile
+        if (local >= 2 &&
+            !mbar_wait(&acc_empty[a], ((local >> 1) - 1) & 1, p.wait, kErrTimeoutAcc)) {
           ok = false;
           break;
         }
         tc_fence_after();
         for (int st = 0; st < nsteps; ++st, ++it) {
           const int s = it % kStages;
-          const uint32_t ph = (it / kStages) & 1;
-          if (!mbar_wait(&full[s], ph, p.wait, kErrTimeoutFull)) {
-            ok = false;
-            break;
-          }
-          const uint32_t a0 = smem_u32(stage_a(s));
-          const uint32_t b0 = smem_u32(stage_b(s));
+          const uint64_t soff = static_cast<uint64_t>((s * L::kStage) >> 4);
           if (st < nk) {
+            const int rg = f & 1;
+            // the stagers arrive only after the slot's operands have landed
+            if (!mbar_wait(&sfready[rg], (f >> 1) & 1, p.wait, kErrTimeoutFull)) {
+              ok = false;
+              break;
+            }
             tc_fence_after();
-            const uint32_t sa = smem_u32(stage_sfa(s));
-            const uint32_t sb = smem_u32(stage_sfb(s));
+            const uint32_t sfr = tmem + L::kSfCol + rg * kSfRegionCols;
             const int nkb = min(4, kblocks - 4 * st);
-            for (int kk = 0; kk < nkb; ++kk) {
-              tmem_cp_32x128b_warpx4(tmem + L::kSfaCol + 4 * kk,
-                                     make_sdesc(sa + kk * 512, 128, 128, kSwzNone));
-#pragma unroll
-              for (int nb = 0; nb < BN / 128; ++nb)
-                tmem_cp_32x128b_warpx4(tmem + L::kSfbCol + (BN / 128) * 4 * kk + 4 * nb,
-                                       make_sdesc(sb + (nb * 4 + kk) * 512, 128, 128, kSwzNone));
-            }
-            for (int kk = 0; kk < nkb; ++kk) {
-              const uint64_t ad = make_sdesc(a0 + kk * 32, 16, 1024, kSwz128);
-              const uint64_t bd = make_sdesc(b0 + kk * 32, 16, 1024, kSwz128);
-              umma_nvfp4(tmem, ad, bd, id_fp4, tmem + L::kSfaCol + 4 * kk,
-                         tmem + L::kSfbCol + (BN / 128) * 4 * kk, (st > 0 || kk > 0) ? 1u : 0u);
-            }
+            for (int kk = 0; kk < nkb; ++kk)
+              umma_nvfp4(acc, da0 + soff + 2 * kk, db0 + soff + 2 * kk, id_fp4, sfr + 4 * kk,
+                         sfr + 16 + 8 * kk, (st > 0 || kk > 0) ? 1u : 0u);
+            umma_commit(&empty[s]);
+            umma_commit(&sffree[rg]);
+            ++f;
           } else {
             if (!mbar_wait(&lrf[s], (lr_par >> s) & 1u, p.wait, kErrTimeoutFull)) {
               ok = false;
@@ -245,123 +274,163 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             lr_par ^= 1u << s;
             tc_fence_after();
-            // packed: A k-steps [0, r/16) hold hi and [2, 2 + r/16) hold lo,
-            // both against B k-steps [0, r/16); unpacked: 4 k-steps per slot
-            const int ksteps = lr_packed ? p.r / 16 : 4;
+            // A k-steps {0, 1} hold hi and {2, 3} lo of the slice's 32
+            // columns, both against B k-steps {0, 1} (r = 16: one of each)
+            const int ksteps = p.r < 32 ? 1 : 2;
             for (int kk = 0; kk < ksteps; ++kk) {
-              const uint64_t bd = make_sdesc(b0 + kk * 32, 16, 1024, kSwz128);
-              umma_f16(tmem, make_sdesc(a0 + kk * 32, 16, 1024, kSwz128), bd, id_f16, 1u);
-              if (lr_packed)
-                umma_f16(tmem, make_sdesc(a0 + (2 + kk) * 32, 16, 1024, kSwz128), bd, id_f16, 1u);
+              umma_f16(acc, da0 + soff + 2 * kk, db0 + soff + 2 * kk, id_f16, 1u);
+              umma_f16(acc, da0 + soff + 2 * (2 + kk), db0 + soff + 2 * kk, id_f16, 1u);
             }
+            umma_commit(&empty[s]);
           }
-          umma_commit(&empty[s]);
-          // the step kStages ahead reuses this slot; if it is a low-rank step,
-          // tell the epilogue when this step's reads of the slot are done
-          if ((it + kStages) % nsteps >= nk) umma_commit(&lrfree[s]);
         }
-        if (ok) umma_commit(acc_full);
+        if (ok) umma_commit(&acc_full[a]);
+      }
+    }
+  } else if (warp < 2 + kStagerWarps) {
+    // ----------------------------------------------------------- stagers ----
+    const int quad = warp & 3;               // TMEM lane quadrant this warp may access
+    const int row = 32 * quad + lane;        // tile row of the low-rank A operand
+    const uint32_t lane_off = static_cast<uint32_t>(32 * quad) << 16;
+    const float gprod = __fmul_rn(*p.gs_a, *p.gs_w);
+    int it = 0, f = 0;
+    uint32_t sf_par = 0;                     // parity of each slot's next full_sf phase
+    bool ok = true;
+    for (int t = blockIdx.x; ok && t < p.tiles; t += gridDim.x) {
+      int m0, n0;
+      tile_coords(t, p.tiles_n, BN, m0, n0);
+      for (int st = 0; ok && st < nsteps; ++st, ++it) {
+        const int s = it % kStages;
+        const uint32_t ph = (it / kStages) & 1;
+        if (st < nk) {
+          // this FP4 step's scales into region rg (its previous user is FP4 step f - 2)
+          const int rg = f & 1;
+          if (f >= 2 && !mbar_wait(&sffree[rg], ((f >> 1) - 1) & 1, p.wait, kErrTimeoutEmpty)) {
+            ok = false;
+            break;
+          }
+          if (!mbar_wait(&full_sf[s], (sf_par >> s) & 1u, p.wait, kErrTimeoutFull)) {
+            ok = false;
+            break;
+          }
+          sf_par ^= 1u << s;
+          tc_fence_after();
+          const uint32_t sfr = tmem + lane_off + L::kSfCol + rg * kSfRegionCols;
+          const int nkb = min(4, kblocks - 4 * st);
+          const uint8_t* sfa = stage_sfa(s);
+          const uint8_t* sfb = stage_sfb(s);
+          for (int kk = 0; kk < nkb; ++kk) {
+            // SFA: column 4kk + j = bytes [4j, 4j + 4) of the block's line `lane`
+            const uint4 va = *reinterpret_cast<const uint4*>(sfa + kk * 512 + lane * 16);
+            tmem_st_32x32b_x4(sfr + 4 * kk, va.x, va.y, va.z, va.w);
+            // SFB: column 16 + 8kk + j holds tile row 32j + lane, which is
+            // weight row n0 + 32j + lane, in block (n0 + 32j + lane)/128 - n0/128
+            uint32_t vb[BN / 32];
+#pragma unroll
+            for (int j = 0; j < BN / 32; ++j) {
+              const int rr = (n0 & 127) + 32 * j;  // row offset from block n0/128
+              vb[j] = *reinterpret_cast<const uint32_t*>(sfb + (rr >> 7) * 2048 + kk * 512 +
+                                                         lane * 16 + ((rr & 127) >> 5) * 4);
+            }
+            tmem_st_32x32b_x4(sfr + 16 + 8 * kk, vb[0], vb[1], vb[2], vb[3]);
+            if constexpr (BN / 32 == 6) tmem_st_32x32b_x2(sfr + 20 + 8 * kk, vb[4], vb[5]);
+          }
+          tmem_st_wait();
+          tc_fence_before();
+          // the MMA thread waits on sfready alone: make it imply the operands too
+          if (!mbar_wait(&full[s], ph, p.wait, kErrTimeoutFull)) {
+            ok = false;
+            break;
+          }
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&sfready[rg]);
+          ++f;
+        } else {
+          // the tile's low-rank A operand, in place over the slot's xl slice
+          if (!mbar_wait(&full[s], ph, p.wait, kErrTimeoutFull)) {
+            ok = false;
+            break;
+          }
+          // this row's 32 fp32 values sit unswizzled in its own 128 bytes:
+          // read them all, then overwrite the same bytes with hi | lo
+          uint8_t* arow = stage_a(s) + row * 128;
+          float w[32];
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            const float4 u = *reinterpret_cast<const float4*>(arow + 16 * q);
+            w[4 * q] = u.x;
+            w[4 * q + 1] = u.y;
+            w[4 * q + 2] = u.z;
+            w[4 * q + 3] = u.w;
+          }
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {  // chunk q: hi of columns 8q..8q+7; chunk 4+q: their lo
+            uint32_t hw[4], lw[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const float t0 = __fmul_rn(w[8 * q + 2 * e], gprod);
+              const float t1 = __fmul_rn(w[8 * q + 2 * e + 1], gprod);
+              const float h0 = __bfloat162float(__float2bfloat16_rn(t0));
+              const float h1 = __bfloat162float(__float2bfloat16_rn(t1));
+              hw[e] = pack_bf16x2(h0, h1);
+              lw[e] = pack_bf16x2(__fsub_rn(t0, h0), __fsub_rn(t1, h1));
+            }
+            *reinterpret_cast<uint4*>(arow + ((q ^ (row & 7)) << 4)) =
+                make_uint4(hw[0], hw[1], hw[2], hw[3]);
+            *reinterpret_cast<uint4*>(arow + (((4 + q) ^ (row & 7)) << 4)) =
+                make_uint4(lw[0], lw[1], lw[2], lw[3]);
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&lrf[s]);
+        }
       }
     }
   } else {
     // ---------------------------------------------------------- epilogue ----
-    const int ew = warp - 2;                 // 0..7
+    const int ew = warp - 2 - kStagerWarps;  // 0..7
     const int quad = warp & 3;               // TMEM lane quadrant this warp may access
-    const int half = ew >> 2;                // which half of BN
-    const int row = 32 * quad + lane;        // tile row == TMEM lane
-    const float gprod = __fmul_rn(*p.gs_a, *p.gs_w);
-    const float alpha = __fdiv_rn(1.0f, gprod);
-    constexpr int kCols = L::kColsPerWarp;
-    int it = 0;
-    uint32_t free_par = 0;                   // parity of each slot's next lrfree phase
+    const int half = ew >> 2;                // which group of 64-column boxes
+    const int box0 = half == 0 ? 0 : L::kBoxes0;
+    const int nbox = half == 0 ? L::kBoxes0 : L::kBoxes - L::kBoxes0;
+    const float alpha = __fdiv_rn(1.0f, __fmul_rn(*p.gs_a, *p.gs_w));
+    uint16_t* bsl = bias_s + ew * (L::kBoxes0 * 64);
+    uint8_t* box = out_s + ew * L::kBoxBytes;
+    uint8_t* brow = box + lane * 128;
     int local = 0;
-    bool ok = true;
-    for (int t = blockIdx.x; ok && t < p.tiles; t += gridDim.x, ++local) {
+    for (int t = blockIdx.x; t < p.tiles; t += gridDim.x, ++local) {
       int m0, n0;
       tile_coords(t, p.tiles_n, BN, m0, n0);
-      const int grow = m0 + row;
-      // (1) this warp's bias slice into its own shared-memory buffer (only
-      // this warp reads it, after the __syncwarp below, and it rewrites it
-      // only after its previous drain finished reading it)
-      uint16_t* bsl = bias_s + ew * kCols;
-      for (int c = lane; c < kCols; c += 32) {
-        const int col = n0 + half * kCols + c;
+      const int a = local & 1;
+      // this warp's bias columns into its own shared-memory slice
+      for (int c = lane; c < nbox * 64; c += 32) {
+        const int col = n0 + 64 * box0 + c;
         bsl[c] = (p.bias && col < p.N) ? p.bias[col] : static_cast<uint16_t>(0);
       }
       __syncwarp();
-      // (2) the low-rank A operand of this tile, into the ring slots of its
-      // low-rank steps (they follow the tile's FP4 steps); one warp per
-      // quadrant writes its 32 rows
-      it += nk;
-      for (int j = 0; j < nlr; ++j, ++it) {
-        const int s = it % kStages;
-        const uint32_t ph = (it / kStages) & 1;
-        (void)ph;
-        if (half != 0) continue;
-        if (it >= kStages) {  // the slot had a previous user: wait until it is done
-          if (!mbar_wait(&lrfree[s], (free_par >> s) & 1u, p.wait, kErrTimeoutEmpty)) {
-            ok = false;
-            break;
-          }
-          free_par ^= 1u << s;
-        }
-        uint8_t* arow = stage_a(s) + row * 128;
-#pragma unroll
-        for (int q = 0; q < 8; ++q) {  // 8 bf16 = one 16-byte chunk
-          // packed: chunks 0-3 = hi of columns 0..31, chunks 4-7 = lo of them;
-          // unpacked: slice j/2, part j%2 (0 = hi, 1 = lo)
-          const int part = lr_packed ? (q >> 2) : (j & 1);
-          const int col0 = lr_packed ? 8 * (q & 3) : 64 * (j >> 1) + 8 * q;
-          float v[8];
-          if (grow < p.M && col0 < p.r) {
-            const float4* src =
-                reinterpret_cast<const float4*>(p.lora + static_cast<size_t>(grow) * p.r + col0);
-            const float4 u0 = src[0], u1 = src[1];
-            const float w8[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
-#pragma unroll
-            for (int e = 0; e < 8; ++e) {
-              const float tv = __fmul_rn(w8[e], gprod);
-              const float hi = __bfloat162float(__float2bfloat16_rn(tv));
-              v[e] = part == 0 ? hi : __fsub_rn(tv, hi);
-            }
-          } else {
-#pragma unroll
-            for (int e = 0; e < 8; ++e) v[e] = 0.0f;
-          }
-          *reinterpret_cast<uint4*>(arow + ((q ^ (row & 7)) << 4)) =
-              make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]),
-                         pack_bf16x2(v[4], v[5]), pack_bf16x2(v[6], v[7]));
-        }
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&lrf[s]);
-      }
-      if (!ok) break;
-      // (3) drain the accumulator: α·acc + bias -> packed bf16 in registers
-      if (!mbar_wait(acc_full, local & 1, p.wait, kErrTimeoutAcc)) {
-        ok = false;
-        break;
-      }
+      if (!mbar_wait(&acc_full[a], (local >> 1) & 1, p.wait, kErrTimeoutAcc)) break;
       tc_fence_after();
-      uint32_t packed[kCols / 2];
-      const uint32_t taddr = tmem + (static_cast<uint32_t>(32 * quad) << 16) + half * kCols;
+      // drain: α·acc + bias -> packed bf16
+      uint32_t packed[L::kBoxes0 * 32];
+      const uint32_t taddr = tmem + (static_cast<uint32_t>(32 * quad) << 16) + a * BN + 64 * box0;
 #pragma unroll
-      for (int c = 0; c < kCols / 16; c += 2) {
-        uint32_t a0[16], a1[16];
-        tmem_ld_32x32b_x16(taddr + c * 16, a0);
-        tmem_ld_32x32b_x16(taddr + (c + 1) * 16, a1);
+      for (int c = 0; c < L::kBoxes0 * 4; c += 2) {  // 16-column chunks, two per load pair
+        if (c >= nbox * 4) break;
+        uint32_t v0[16], v1[16];
+        tmem_ld_32x32b_x16(taddr + c * 16, v0);
+        tmem_ld_32x32b_x16(taddr + (c + 1) * 16, v1);
         tmem_ld_wait();
 #pragma unroll
         for (int u = 0; u < 2; ++u) {
-          const uint32_t* a = u ? a1 : a0;
+          const uint32_t* av = u ? v1 : v0;
           const uint4* b4 = reinterpret_cast<const uint4*>(bsl + (c + u) * 16);
           const uint4 bb0 = b4[0], bb1 = b4[1];
           const uint32_t bw[8] = {bb0.x, bb0.y, bb0.z, bb0.w, bb1.x, bb1.y, bb1.z, bb1.w};
 #pragma unroll
           for (int e = 0; e < 8; ++e) {
-            const float lo = __fadd_rn(__fmul_rn(__uint_as_float(a[2 * e]), alpha),
+            const float lo = __fadd_rn(__fmul_rn(__uint_as_float(av[2 * e]), alpha),
                                        __uint_as_float(bw[e] << 16));
-            const float hi = __fadd_rn(__fmul_rn(__uint_as_float(a[2 * e + 1]), alpha),
+            const float hi = __fadd_rn(__fmul_rn(__uint_as_float(av[2 * e + 1]), alpha),
                                        __uint_as_float(bw[e] & 0xFFFF0000u));
             packed[(c + u) * 8 + e] = pack_bf16x2(lo, hi);
           }
@@ -369,31 +438,43 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(acc_empty);   // the MMA may start the next tile
-      // (4) store y (overlaps the next tile's mainloop)
-      const int colb = n0 + half * kCols;
-      if (grow < p.M) {
-        uint4* dst = reinterpret_cast<uint4*>(p.y + static_cast<size_t>(grow) * p.ldy + colb);
+      if (lane == 0) mbar_arrive(&acc_empty[a]);  // the MMAs may refill this accumulator
+      // store: one 32 x 64 staging box per 64 columns, 128-byte swizzle
 #pragma unroll
-        for (int q = 0; q < kCols / 8; ++q)
-          if (colb + 8 * q < p.N)
-            dst[q] = make_uint4(packed[4 * q], packed[4 * q + 1], packed[4 * q + 2], packed[4 * q + 3]);
+      for (int j = 0; j < L::kBoxes0; ++j) {
+        if (j >= nbox) break;
+        if (lane == 0) bulk_wait_group_read<0>();  // the previous box has left shared memory
+        __syncwarp();
+#pragma unroll
+        for (int q = 0; q < 8; ++q)
+          *reinterpret_cast<uint4*>(brow + ((q ^ (lane & 7)) << 4)) =
+              make_uint4(packed[32 * j + 4 * q], packed[32 * j + 4 * q + 1],
+                         packed[32 * j + 4 * q + 2], packed[32 * j + 4 * q + 3]);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          tma_store_2d(&tmap_y, box, n0 + 64 * (box0 + j), m0 + 32 * quad);
+          bulk_commit_group();
+        }
       }
     }
+    if (lane == 0) bulk_wait_group<0>();  // all of this warp's stores are complete
   }
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, L::kTmemCols);
+    tmem_dealloc(tmem, 512);
   }
 }
 
 template <int BN>
 svdq_status launch_bn(const LaunchCtx& ctx, const CUtensorMap& ta, const CUtensorMap& tb,
-                      const CUtensorMap& tl, GemmParams p) {
+                      const CUtensorMap& tl, const CUtensorMap& ty, const CUtensorMap& tr,
+                      GemmParams p) {
   using L = Layout<BN>;
-  const size_t smem = 1024 + static_cast<size_t>(L::kRing) + L::kBias + 8 * (4 * kStages + 2) + 16;
+  const size_t smem = 1024 + static_cast<size_t>(L::kRing) + kEpiWarps * L::kBoxBytes + L::kBias +
+                      8 * (4 * kStages + 8) + 16;
   static bool attr_done[64] = {};
   if (!attr_done[ctx.device & 63]) {
     cudaFuncSetAttribute(w4a4_gemm_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -403,7 +484,7 @@ svdq_status launch_bn(const LaunchCtx& ctx, const CUtensorMap& ta, const CUtenso
   p.tiles_n = (p.N + BN - 1) / BN;
   p.tiles = p.tiles_n * ((p.M + kBM - 1) / kBM);
   const int grid = std::min(p.tiles, ctx.num_sms);
-  w4a4_gemm_kernel<BN><<<grid, kThreads, smem, ctx.stream>>>(ta, tb, tl, p);
+  w4a4_gemm_kernel<BN><<<grid, kThreads, smem, ctx.stream>>>(ta, tb, tl, ty, tr, p);
   return check_launch("w4a4_gemm_kernel");
 }
 
@@ -414,8 +495,8 @@ svdq_status launch_w4a4_gemm(const LaunchCtx& ctx, const uint8_t* q_act, const u
                              const uint8_t* sf_w, const float* w_gscale, const void* L2t, int r,
                              const void* bias, int64_t M, int64_t N, int64_t K, void* y,
                              int64_t ldy) {
-  const int bn = (N % 256 == 0) ? 256 : 128;
-  CUtensorMap ta{}, tb{}, tl{};
+  const int bn = (N % 192 == 0) ? 192 : 128;
+  CUtensorMap ta{}, tb{}, tl{}, ty{}, tr{};
   if (!make_tmap_2d(&ta, q_act, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, M, K / 2, K / 2, kBM, kBKBytes,
                     128))
     return SVDQ_ERR_CUDA;
@@ -428,6 +509,17 @@ svdq_status launch_w4a4_gemm(const LaunchCtx& ctx, const uint8_t* q_act, const u
   } else {
     tl = ta;
   }
+  if (r > 0) {
+    // xl [M, r] fp32 in 128-row x 32-column boxes (zero past M and r)
+    if (!make_tmap_2d(&tr, lora_act, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, M, r,
+                      static_cast<uint64_t>(r) * 4, kBM, 32, 0))
+      return SVDQ_ERR_CUDA;
+  } else {
+    tr = ta;
+  }
+  if (!make_tmap_2d(&ty, y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, M, N, static_cast<uint64_t>(ldy) * 2,
+                    32, 64, 128))
+    return SVDQ_ERR_CUDA;
   GemmParams p{};
   p.M = static_cast<int>(M);
   p.N = static_cast<int>(N);
@@ -437,13 +529,11 @@ svdq_status launch_w4a4_gemm(const LaunchCtx& ctx, const uint8_t* q_act, const u
   p.sf_w = sf_w;
   p.gs_a = act_gscale;
   p.gs_w = w_gscale;
-  p.lora = lora_act;
   p.bias = static_cast<const uint16_t*>(bias);
-  p.y = static_cast<uint16_t*>(y);
-  p.ldy = ldy;
   p.fault = ctx.fault_flags;
   p.wait = WaitCfg{ctx.timeout_ns, ctx.err_word};
-  return bn == 256 ? launch_bn<256>(ctx, ta, tb, tl, p) : launch_bn<128>(ctx, ta, tb, tl, p);
+  return bn == 192 ? launch_bn<192>(ctx, ta, tb, tl, ty, tr, p)
+                   : launch_bn<128>(ctx, ta, tb, tl, ty, tr, p);
 }
 
 }  // namespace svdq

@@ -30,6 +30,10 @@ bool make_tmap_2d(CUtensorMap* map, const void* base, CUtensorMapDataType dtype,
 svdq_status fail(svdq_status st, const char* fmt, ...);
 svdq_status check_launch(const char* what);
 
+// Shared memory the quantize kernel needs for a [*, K] activation at rank r
+// (the API rejects shapes above the 227 KB per-CTA limit before launching).
+size_t quantize_smem_bytes(int64_t K, int r);
+
 // Kernel launchers (one per translation unit).  Arguments are validated.
 svdq_status launch_quantize_act(const LaunchCtx& ctx, const void* x, int64_t M, int64_t K,
                                 int64_t ldx, const float* smooth_s, const void* L1t, int r,

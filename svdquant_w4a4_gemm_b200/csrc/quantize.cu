@@ -12,20 +12,25 @@
 // (one persistent CTA per SM), so the memory pipeline never drains between
 // work items and the load is balanced to one sub-tile.
 //   warp 0       TMA producer: x sub-tiles and the matching 64-column slices
-//                of L1ᵀ into a kStages-deep shared-memory ring; its lanes
-//                also compute RN(1/s) for the slot's 64 columns.
+//                of L1ᵀ into a kStages-deep shared-memory ring.  The first
+//                kStages loads are issued before the CTA-wide set-up, while
+//                the other warps compute RN(1/s) once for every column this
+//                CTA's range touches.
 //   warp 1       TMEM owner; one thread issues the down-projection as
 //                tcgen05 kind::f16 MMAs (M = 128, N = r, K = 16 each) from
 //                the quantized tile's bf16(x̂) and the L1ᵀ slice into a TMEM
 //                accumulator; a new accumulator (of two) per run of
 //                sub-tiles in the same 128-row block ("segment").
-//   warps 2-9    quantizers: one thread = one row x 32 columns = two
-//                16-element groups: x̂ = x·inv_s, group max, E4M3 scale
-//                (cvt.rn.satfinite.e4m3x2), E2M1 codes (cvt.rn.satfinite
-//                .e2m1x2, sign bit copied), a 16-byte code store, a 2-byte
-//                scale store into the 128x4 block layout, and bf16(x̂)
-//                written back over the tile for the MMA.
-//   warps 10-13  epilogue: when a segment's accumulator is complete, TMEM ->
+//   warps 2-17   quantizers: one thread = one row x one 16-element group
+//                (a warp = 8 rows x the tile's 4 groups, so four consecutive
+//                lanes write 32 contiguous code bytes and the row's 4 scale
+//                bytes): x̂ = x·inv_s, group max, E4M3 scale
+//                (cvt.rn.satfinite.e4m3x2; RN(gs / scale) from a per-CTA
+//                table of the 127 scale codes), E2M1 codes (cvt.rn.satfinite
+//                .e2m1x2), an 8-byte code store, a 1-byte scale store into
+//                the 128x4 block layout, and bf16(x̂) written back over the
+//                tile for the MMA.
+//   warps 18-21  epilogue: when a segment's accumulator is complete, TMEM ->
 //                registers -> float4 atomics into xl (zeroed beforehand:
 //                a row block's K range can span several CTAs), then release
 //                the accumulator.
@@ -42,7 +47,7 @@ namespace {
 constexpr int kBM = 128;
 constexpr int kSubK = 64;
 constexpr int kStages = 4;
-constexpr int kQuantWarps = 8;
+constexpr int kQuantWarps = 16;
 constexpr int kEpiWarps = 4;
 constexpr int kThreads = 32 * (2 + kQuantWarps + kEpiWarps);
 constexpr uint32_t kXTileBytes = kBM * kSubK * 2;
@@ -68,15 +73,6 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&h);
 }
 
-// Copy each value's sign into bit 3 of its nibble (a value that rounds to
-// zero keeps its sign: E2M1 code 0x8 for negative inputs).
-__device__ __forceinline__ uint32_t e2m1_signs(const float (&v)[8]) {
-  uint32_t s = 0;
-#pragma unroll
-  for (int i = 0; i < 8; ++i) s |= (__float_as_uint(v[i]) >> 31) << (4 * i + 3);
-  return s;
-}
-
 __device__ __forceinline__ float tensor_scale_from_amax(float amax) {
   return amax > 0.0f ? __fdiv_rn(2688.0f, amax) : 1.0f;
 }
@@ -96,8 +92,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t l1_bytes = static_cast<uint32_t>(p.r) * 128u;
   uint8_t* xs = base;
   uint8_t* ls = xs + kStages * kXTileBytes;
-  float* inv_st = reinterpret_cast<float*>(ls + kStages * l1_bytes);  // [kStages][64]
-  uint64_t* full = reinterpret_cast<uint64_t*>(inv_st + kStages * kSubK);
+  float* inv_s = reinterpret_cast<float*>(ls + kStages * l1_bytes);   // [K], touched columns
+  float* gs_over_d = inv_s + p.K;                                     // [128] by E4M3 code
+  uint64_t* full = reinterpret_cast<uint64_t*>(gs_over_d + 128);
   uint64_t* qdone = full + kStages;
   uint64_t* empty = qdone + kStages;
   uint64_t* acc_full = empty + kStages;  // [2]
@@ -111,7 +108,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   int u0, u1;
   unit_range(p.units, u0, u1);
 
-  if (threadIdx.x == 0) {
+  // Warp 0 sets up the barriers and issues the first kStages loads right
+  // away; the rest of the CTA fills the RN(1/s) and RN(gs/scale) tables in
+  // the meantime.  Nobody else touches a barrier before the __syncthreads.
+  if (warp == 0 && lane == 0) {
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&qdone[s], kQuantWarps);
@@ -122,14 +122,39 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&acc_empty[b], kEpiWarps);
     }
     fence_mbar_init();
-  }
-  if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tmap_x);
     if (has_lr) tma_prefetch_desc(&tmap_l1);
+    for (int u = u0; u < min(u1, u0 + kStages); ++u) {
+      const int s = u - u0;
+      const int rb = u / kblocks, kb = u % kblocks;
+      mbar_arrive_expect_tx(&full[s], kXTileBytes + (has_lr ? l1_bytes : 0u));
+      tma_load_2d(xs + s * kXTileBytes, &tmap_x, &full[s], kb * kSubK, rb * kBM);
+      if (has_lr) tma_load_2d(ls + s * l1_bytes, &tmap_l1, &full[s], kb * kSubK, 0);
+    }
+  }
+  if (warp != 0) {
+    // RN(1/s) for the columns of every sub-tile in [u0, u1): the whole K if
+    // the range covers it, else per sub-tile (repeats write the same value)
+    const int t = threadIdx.x - 32, nt = kThreads - 32;
+    if (u1 - u0 >= kblocks) {
+      for (int j = t; j < p.K; j += nt) inv_s[j] = p.smooth_s ? __fdiv_rn(1.0f, p.smooth_s[j]) : 1.0f;
+    } else {
+      for (int j = t; j < (u1 - u0) * kSubK; j += nt) {
+        const int col = ((u0 + j / kSubK) % kblocks) * kSubK + j % kSubK;
+        inv_s[col] = p.smooth_s ? __fdiv_rn(1.0f, p.smooth_s[col]) : 1.0f;
+      }
+    }
   }
   if (warp == 1 && has_lr) {
     tmem_alloc(tmem_slot, tmem_cols);
     tmem_relinquish();
+  }
+  // RN(gs / dec(sf)) for every finite E4M3 scale code (0 for the zero
+  // scale): one IEEE division per code per CTA instead of one per group
+  const float gs = p.gs_in ? *p.gs_in : tensor_scale_from_amax(*p.amax_src);
+  if (threadIdx.x < 128) {
+    const float d = e4m3_to_f32(threadIdx.x);
+    gs_over_d[threadIdx.x] = (d == 0.0f || threadIdx.x == 127) ? 0.0f : __fdiv_rn(gs, d);
   }
   tc_fence_before();
   __syncthreads();
@@ -138,34 +163,23 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == 0) {
     // ------------------------------------------------------- producer ----
-    int issued = 0;
-    for (int u = u0; u < u1; ++u) {
-      const int i = u - u0;
-      const int s = i % kStages;
-      const uint32_t ph = (i / kStages) & 1;
-      int ok = 1;
-      if (lane == 0) ok = mbar_wait(&empty[s], ph ^ 1, p.wait, kErrTimeoutEmpty) ? 1 : 0;
-      if (!__shfl_sync(0xffffffffu, ok, 0)) break;
-      const int rb = u / kblocks, kb = u % kblocks;
-      // RN(1/s) of this slot's 64 columns, published by the arrive below
-      float2 iv = make_float2(1.0f, 1.0f);
-      if (p.smooth_s) {
-        const float2 sv = *reinterpret_cast<const float2*>(p.smooth_s + kb * kSubK + 2 * lane);
-        iv = make_float2(__fdiv_rn(1.0f, sv.x), __fdiv_rn(1.0f, sv.y));
-      }
-      reinterpret_cast<float2*>(inv_st + s * kSubK)[lane] = iv;
-      __syncwarp();
-      if (lane == 0) {
+    if (lane == 0) {
+      int issued = min(u1 - u0, kStages);  // issued before the set-up sync
+      for (int u = u0 + kStages; u < u1; ++u) {
+        const int i = u - u0;
+        const int s = i % kStages;
+        const uint32_t ph = (i / kStages) & 1;
+        if (!mbar_wait(&empty[s], ph ^ 1, p.wait, kErrTimeoutEmpty)) break;
+        const int rb = u / kblocks, kb = u % kblocks;
         mbar_arrive_expect_tx(&full[s], kXTileBytes + (has_lr ? l1_bytes : 0u));
         tma_load_2d(xs + s * kXTileBytes, &tmap_x, &full[s], kb * kSubK, rb * kBM);
         if (has_lr) tma_load_2d(ls + s * l1_bytes, &tmap_l1, &full[s], kb * kSubK, 0);
+        issued = i + 1;
       }
-      issued = i + 1;
-    }
-    // never leave the CTA with a copy still landing in its shared memory
-    if (lane == 0)
+      // never leave the CTA with a copy still landing in its shared memory
       for (int i = max(0, issued - kStages); i < issued; ++i)
         mbar_wait(&full[i % kStages], (i / kStages) & 1, p.wait, kErrTimeoutDrain);
+    }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA ----
     if (has_lr && lane == 0) {
@@ -204,14 +218,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp < 2 + kQuantWarps) {
     // ------------------------------------------------------ quantizers ----
     const int qw = warp - 2;
-    const int row = 32 * (qw & 3) + lane;  // row within the tile
-    const int half = qw >> 2;              // which 32 of the 64 columns
-    float gs;
-    if (p.gs_in) {
-      gs = *p.gs_in;
-    } else {
-      gs = tensor_scale_from_amax(*p.amax_src);
-    }
+    const int row = 8 * qw + (lane >> 2);  // row within the tile
+    const int g = lane & 3;                // which 16-element group of the 64 columns
     if (p.gs_copy && blockIdx.x == 0 && threadIdx.x == 64) *p.gs_copy = gs;
     const size_t kbytes = static_cast<size_t>(p.K) / 2;
     for (int u = u0; u < u1; ++u) {
@@ -222,69 +230,51 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int rb = u / kblocks, kb = u % kblocks;
       const int grow = rb * kBM + row;
       uint8_t* trow = xs + s * kXTileBytes + row * 128;
-      const int kc0 = kb * kSubK + 32 * half;  // first column of this thread
-      const float* inv_s = inv_st + s * kSubK + 32 * half;
-      uint4 v[4];
+      const int kc0 = kb * kSubK + 16 * g;  // first column of this thread's group
+      uint8_t* c0p = trow + (((2 * g) ^ (row & 7)) << 4);
+      uint8_t* c1p = trow + (((2 * g + 1) ^ (row & 7)) << 4);
+      const uint4 v0 = *reinterpret_cast<const uint4*>(c0p);
+      const uint4 v1 = *reinterpret_cast<const uint4*>(c1p);
+      const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+      float xh[16];
+      const float4* is4 = reinterpret_cast<const float4*>(inv_s + kc0);
 #pragma unroll
-      for (int j = 0; j < 4; ++j)
-        v[j] = *reinterpret_cast<const uint4*>(trow + (((4 * half + j) ^ (row & 7)) << 4));
-      uint32_t codes[4];
-      uint32_t sfb[2];
-      uint4 back[4];
-#pragma unroll
-      for (int g = 0; g < 2; ++g) {
-        const uint32_t w[8] = {v[2 * g].x,     v[2 * g].y,     v[2 * g].z,     v[2 * g].w,
-                               v[2 * g + 1].x, v[2 * g + 1].y, v[2 * g + 1].z, v[2 * g + 1].w};
-        float xh[16];
-        const float4* is4 = reinterpret_cast<const float4*>(inv_s + 16 * g);
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const float4 iv = is4[q];
-          xh[4 * q + 0] = __fmul_rn(bf16lo(w[2 * q]), iv.x);
-          xh[4 * q + 1] = __fmul_rn(bf16hi(w[2 * q]), iv.y);
-          xh[4 * q + 2] = __fmul_rn(bf16lo(w[2 * q + 1]), iv.z);
-          xh[4 * q + 3] = __fmul_rn(bf16hi(w[2 * q + 1]), iv.w);
-        }
-        float amax = 0.0f;
-#pragma unroll
-        for (int e = 0; e < 16; ++e) amax = fmaxf(amax, fabsf(xh[e]));
-        const float t = __fmul_rn(__fdiv_rn(amax, 6.0f), gs);
-        const uint32_t sf = cvt_e4m3(t);
-        const float d = e4m3_to_f32(sf);
-        const float inv = d == 0.0f ? 0.0f : __fdiv_rn(gs, d);
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          float q8[8], x8[8];
-#pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            x8[e] = xh[8 * h + e];
-            q8[e] = __fmul_rn(x8[e], inv);
-          }
-          codes[2 * g + h] = cvt_e2m1x8(q8) | e2m1_signs(x8);
-        }
-        sfb[g] = sf;
-        if (has_lr) {
-#pragma unroll
-          for (int h = 0; h < 2; ++h)
-            back[2 * g + h] = make_uint4(pack_bf16x2(xh[8 * h + 0], xh[8 * h + 1]),
-                                         pack_bf16x2(xh[8 * h + 2], xh[8 * h + 3]),
-                                         pack_bf16x2(xh[8 * h + 4], xh[8 * h + 5]),
-                                         pack_bf16x2(xh[8 * h + 6], xh[8 * h + 7]));
-        }
+      for (int q = 0; q < 4; ++q) {
+        const float4 iv = is4[q];
+        xh[4 * q + 0] = __fmul_rn(bf16lo(w[2 * q]), iv.x);
+        xh[4 * q + 1] = __fmul_rn(bf16hi(w[2 * q]), iv.y);
+        xh[4 * q + 2] = __fmul_rn(bf16lo(w[2 * q + 1]), iv.z);
+        xh[4 * q + 3] = __fmul_rn(bf16hi(w[2 * q + 1]), iv.w);
       }
-      if (grow < p.M) {
-        *reinterpret_cast<uint4*>(p.q_out + static_cast<size_t>(grow) * kbytes + kc0 / 2) =
-            make_uint4(codes[0], codes[1], codes[2], codes[3]);
+      float amax = 0.0f;
+#pragma unroll
+      for (int e = 0; e < 16; ++e) amax = fmaxf(amax, fabsf(xh[e]));
+      const float t = __fmul_rn(__fdiv_rn(amax, 6.0f), gs);
+      const uint32_t sf = cvt_e4m3(t);
+      const float inv = gs_over_d[sf & 127u];  // RN(gs / dec(sf)); 0 for a zero scale
+      // cvt.rn.satfinite.e2m1x2 rounds ties to even and keeps the sign of a
+      // value that rounds to zero (code 0x8), as the format requires; the
+      // bit-exact tests hold it to that
+      uint32_t codes[2];
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        float q8[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) q8[e] = __fmul_rn(xh[8 * h + e], inv);
+        codes[h] = cvt_e2m1x8(q8);
       }
+      if (grow < p.M)
+        *reinterpret_cast<uint2*>(p.q_out + static_cast<size_t>(grow) * kbytes + kc0 / 2) =
+            make_uint2(codes[0], codes[1]);
       // rows past M inside the last 128-row block hold zero-filled x, so
       // their scales are written as the zero padding the layout requires
-      *reinterpret_cast<uint16_t*>(p.sf_out + (static_cast<size_t>(rb) * kblocks + kb) * 512 +
-                                   (row & 31) * 16 + (row >> 5) * 4 + 2 * half) =
-          static_cast<uint16_t>(sfb[0] | (sfb[1] << 8));
+      p.sf_out[(static_cast<size_t>(rb) * kblocks + kb) * 512 + (row & 31) * 16 + (row >> 5) * 4 + g] =
+          static_cast<uint8_t>(sf);
       if (has_lr) {
-#pragma unroll
-        for (int j = 0; j < 4; ++j)
-          *reinterpret_cast<uint4*>(trow + (((4 * half + j) ^ (row & 7)) << 4)) = back[j];
+        *reinterpret_cast<uint4*>(c0p) = make_uint4(pack_bf16x2(xh[0], xh[1]), pack_bf16x2(xh[2], xh[3]),
+                                                    pack_bf16x2(xh[4], xh[5]), pack_bf16x2(xh[6], xh[7]));
+        *reinterpret_cast<uint4*>(c1p) = make_uint4(pack_bf16x2(xh[8], xh[9]), pack_bf16x2(xh[10], xh[11]),
+                                                    pack_bf16x2(xh[12], xh[13]), pack_bf16x2(xh[14], xh[15]));
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) mbar_arrive(&qdone[s]);
@@ -374,12 +364,15 @@ __global__ void act_scale_finalize_kernel(float* gs) {
 
 }  // namespace
 
+size_t quantize_smem_bytes(int64_t K, int r) {
+  return 1024 + kStages * (kXTileBytes + static_cast<size_t>(r) * 128) + static_cast<size_t>(K) * 4 +
+         128 * 4 + 8 * (3 * kStages + 4) + 16;
+}
+
 svdq_status launch_quantize_act(const LaunchCtx& ctx, const void* x, int64_t M, int64_t K,
                                 int64_t ldx, const float* smooth_s, const void* L1t, int r,
                                 const float* act_gscale, float* act_gscale_out, uint8_t* q_out,
                                 uint8_t* sf_out, float* lora_out) {
-  if (smooth_s && (reinterpret_cast<uintptr_t>(smooth_s) & 7))
-    return fail(SVDQ_ERR_MISALIGNED, "smooth_s must be 8-byte aligned");
   CUtensorMap tx{}, tl{};
   if (!make_tmap_2d(&tx, x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, M, K, ldx * 2, kBM, kSubK, 128))
     return SVDQ_ERR_CUDA;
@@ -414,8 +407,7 @@ svdq_status launch_quantize_act(const LaunchCtx& ctx, const void* x, int64_t M, 
                                                   smooth_s, reinterpret_cast<unsigned*>(act_gscale_out));
     if (svdq_status e = check_launch("act_amax_kernel")) return e;
   }
-  const size_t smem = 1024 + kStages * (kXTileBytes + static_cast<size_t>(r) * 128 + kSubK * 4) +
-                      8 * (3 * kStages + 4) + 16;
+  const size_t smem = quantize_smem_bytes(K, r);
   static bool attr_done[64] = {};
   if (!attr_done[ctx.device & 63]) {
     cudaFuncSetAttribute(quantize_act_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
