@@ -13,38 +13,38 @@
 // Persistent kernel: one CTA per SM walks 128 x BN output tiles (BN = 192
 // when N is a multiple of 192, else 128).  Tensor memory holds two fp32
 // accumulators (the epilogue drains one while the MMAs fill the other) and
-// two scale-factor regions (the stagers fill one while the MMAs read the
-// other): 2·BN + 2·48 <= 512 columns.
-//   warp 0      producer: per FP4 step (256 K) bulk copies of the matching
-//               128x4 scale blocks (first, on their own barrier, so that the
-//               stagers can start while the operands land), then TMA of
-//               packed A (128 rows x 128 B) and B (BN rows x 128 B) with
-//               128-byte swizzle; per low-rank step (32 of the r columns)
-//               TMA of the L2ᵀ slice and of the tile's fp32 xl slice (into
-//               the A slot).  One kStages-deep ring.
-//   warp 1      TMEM owner and MMA issuer (one thread): four block-scaled
+// a ring of scale-factor regions (the stagers fill regions ahead of the MMAs
+// that read them): 3 regions of 40 columns at BN = 192, 8 of 32 at BN = 128.
+//   warps 0-1   producers (slot s of the kStages-deep ring belongs to warp
+//               s % 2): per FP4 step (256 K) bulk copies of the step's
+//               128x4 scale blocks (on their own barrier, so the stagers can
+//               start while the operands land), then TMA of packed A (128
+//               rows x 128 B) and B (BN rows x 128 B) with 128-byte swizzle; per
+//               low-rank step (32 of the r columns) TMA of the L2ᵀ slice and
+//               of the tile's fp32 xl slice (into the A slot).  A thread that
+//               issues copies spends a few hundred cycles per barrier round,
+//               so two threads share the work.
+//   warp 2      TMEM owner and MMA issuer (one thread): four block-scaled
 //               MMAs (K = 64 each) per FP4 step, then the low-rank kind::f16
 //               MMAs, into the tile's accumulator; tcgen05.commit frees ring
 //               slots and scale regions and, at the end of a tile, hands the
-//               accumulator to the epilogue.
-//   warps 2-5   stagers, one per 32-lane TMEM quadrant.  Per FP4 step they
-//               move the step's E4M3 scales from shared memory into a scale
-//               region with tcgen05.st, every quadrant holding the same
-//               copy (lane l, column j: the 4 scales of row 32j + l per
-//               64-K block, the order the block-scaled MMA reads).  Stores
-//               from registers run beside the MMAs; a shared-to-TMEM copy
-//               issued by the MMA thread would queue behind them.  Per
-//               low-rank step they turn the slot's xl slice in place into
-//               the low-rank A operand: 32 columns of hi and 32 of lo (bf16
-//               of xl·gs_a·gs_w and of its remainder), swizzled by hand.
-//               The MMA thread waits on one barrier per step (the stagers'),
-//               and keeps nothing but MMA issue on its path: the tensor pipe
-//               holds only about one MMA ahead, so any latency in the issuing
-//               thread shows up as idle tensor cycles.
-//   warps 6-13  epilogue, two per quadrant: TMEM -> registers (α·acc + bias
-//               -> bf16), release the accumulator, then 32 x 64 staging
-//               boxes in shared memory and TMA stores of y (full-line
-//               writes, clipped at the M and N edges).
+//               accumulator to the epilogue.  It waits on one barrier per
+//               step and does nothing else: the tensor pipe holds about one
+//               MMA ahead, so latency in the issuing thread idles it.
+//   warps 3-6   stagers, one per 32-lane TMEM quadrant.  Per FP4 step they
+//               read the step's E4M3 scales from the ring slot and write them
+//               into a scale region with tcgen05.st, every quadrant holding
+//               the same copy (lane l, column j: the 4 scales of row 32j + l
+//               per 64-K block, the order the block-scaled MMA reads).  Stores from registers run
+//               beside the MMAs; a shared-to-TMEM copy issued by the MMA
+//               thread would queue behind them.  Per low-rank step they turn
+//               the slot's xl slice in place into the low-rank A operand: 32
+//               columns of hi and 32 of lo (bf16 of xl·gs_a·gs_w and of its
+//               remainder), swizzled by hand.
+//   warps 7-10  epilogue, one per quadrant: per 64-column box, TMEM ->
+//               registers (α·acc + bias -> bf16) -> a 32 x 64 staging box in
+//               shared memory -> TMA store (full-line writes, clipped at the
+//               M and N edges); then release the accumulator.
 #include "internal.h"
 #include "ptx.cuh"
 
@@ -53,12 +53,15 @@ namespace {
 
 constexpr int kBM = 128;
 constexpr int kBKBytes = 128;  // 256 FP4 elements per FP4 step and row
-constexpr int kStages = 4;
+constexpr int kStages = 4;                 // ring slots
+constexpr int kProducers = 2;              // producer warps; slot s belongs to producer s % 2
+constexpr int kMmaWarp = kProducers;
 constexpr int kStagerWarps = 4;
-constexpr int kEpiWarps = 8;
-constexpr int kThreads = 32 * (2 + kStagerWarps + kEpiWarps);
+constexpr int kEpiWarps = 4;
+// 11 warps: at most 3 per SM sub-partition, so up to 168 registers a thread
+constexpr int kThreads = 32 * (kProducers + 1 + kStagerWarps + kEpiWarps);
 constexpr uint32_t kATileBytes = kBM * kBKBytes;  // 16 KB
-constexpr uint32_t kSfRegionCols = 48;            // SFA 4 x 4 + SFB 4 x 8 columns
+constexpr int kMaxRegions = 8;
 
 struct GemmParams {
   int M, N, K, r;
@@ -81,16 +84,23 @@ template <int BN>
 struct Layout {
   static constexpr uint32_t kB = BN * kBKBytes;          // B tile bytes
   static constexpr uint32_t kSfa = 4 * 512;              // 4 K-blocks x 128 rows
-  static constexpr uint32_t kSfb = 2 * 4 * 512;          // up to two 128-row blocks
+  static constexpr uint32_t kSfb = (BN > 128 ? 2 : 1) * 4 * 512;  // one or two 128-row blocks
   static constexpr uint32_t kStage = kATileBytes + kB + kSfa + kSfb;
   static constexpr uint32_t kRing = kStages * kStage;
   static constexpr int kBoxes = BN / 64;                 // 64-column store boxes per tile
-  static constexpr int kBoxes0 = (kBoxes + 1) / 2;       // boxes of the half-0 epilogue warps
   static constexpr uint32_t kBoxBytes = 32 * 128;        // 32 rows x 64 bf16
-  static constexpr uint32_t kBias = kEpiWarps * kBoxes0 * 64 * 2;
+  static constexpr uint32_t kBias = kEpiWarps * BN * 2;  // per-warp bias copies
+  // A scale region holds one FP4 step's scales: SFA (4 columns per 64-K
+  // block) at 4kk, SFB (BN/32 columns per block) at 16 + (BN/32)kk.  As
+  // many regions as fit after the two accumulators: a region is rewritten
+  // only after the MMAs that read it completed, and that completion reaches
+  // the stagers about two steps after the MMAs were issued.
+  static constexpr uint32_t kSfbCols = BN / 32;
+  static constexpr uint32_t kSfRegionCols = 16 + 4 * kSfbCols;
   static constexpr uint32_t kSfCol = 2 * BN;             // first scale-region column
+  static constexpr int kRegions = (512 - 2 * BN) / kSfRegionCols;
   static_assert(kStage % 1024 == 0, "stage must keep 1 KB alignment");
-  static_assert(2 * BN + 2 * kSfRegionCols <= 512, "TMEM budget");
+  static_assert(kRegions >= 3 && kRegions <= kMaxRegions, "TMEM budget");
   static_assert(BN % 64 == 0 && BN <= 256, "tile width");
 };
 
@@ -114,12 +124,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* out_s = base + L::kRing;                                     // [kEpiWarps][box]
   uint16_t* bias_s = reinterpret_cast<uint16_t*>(out_s + kEpiWarps * L::kBoxBytes);
   uint64_t* full = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(bias_s) + L::kBias);
-  uint64_t* full_sf = full + kStages;    // the slot's scale blocks landed (FP4 steps only)
+  uint64_t* full_sf = full + kStages;    // the slot's scale blocks landed (FP4 steps)
   uint64_t* empty = full_sf + kStages;
   uint64_t* lrf = empty + kStages;       // low-rank A written, per ring slot
-  uint64_t* sfready = lrf + kStages;     // [2] scale region written (and the slot's operands landed)
-  uint64_t* sffree = sfready + 2;        // [2] scale region read by its MMAs
-  uint64_t* acc_full = sffree + 2;       // [2]
+  uint64_t* sfready = lrf + kStages;     // [kRegions] scale region written (and the slot's operands landed)
+  uint64_t* sffree = sfready + kMaxRegions;  // [kRegions] scale region read by its MMAs
+  uint64_t* acc_full = sffree + kMaxRegions; // [2]
   uint64_t* acc_empty = acc_full + 2;    // [2]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
   auto stage_a = [&](int s) { return base + s * L::kStage; };
@@ -133,7 +143,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int kblocks = p.K / 64;              // 64-element K blocks (one MMA each)
   const int nk = (kblocks + 3) / 4;          // FP4 steps per tile (the last may be short)
   const int nsteps = nk + nlr;               // ring steps per tile
-  const int nb_total = (p.N + 127) / 128;    // 128-row blocks of the weight scales
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
@@ -142,22 +151,24 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&empty[s], 1);
       mbar_init(&lrf[s], kStagerWarps);
     }
-    for (int b = 0; b < 2; ++b) {
+    for (int b = 0; b < L::kRegions; ++b) {
       mbar_init(&sfready[b], kStagerWarps);
       mbar_init(&sffree[b], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
       mbar_init(&acc_full[b], 1);
       mbar_init(&acc_empty[b], kEpiWarps);
     }
     fence_mbar_init();
   }
-  if (warp == 0 && lane == 0) {
+  if (warp == kMmaWarp && lane == 0) {
     tma_prefetch_desc(&tmap_a);
     tma_prefetch_desc(&tmap_b);
     if (p.r > 0) tma_prefetch_desc(&tmap_l2);
     if (p.r > 0) tma_prefetch_desc(&tmap_lr);
     tma_prefetch_desc(&tmap_y);
   }
-  if (warp == 1) {
+  if (warp == kMmaWarp) {
     tmem_alloc(tmem_slot, 512);
     tmem_relinquish();
   }
@@ -166,22 +177,21 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 0) {
-    // ------------------------------------------------------- producer ----
+  if (warp < kProducers) {
+    // ------------------------------------------------------ producers ----
     if (lane == 0) {
       int it = 0;              // ring step counter (continues across tiles)
-      uint32_t used = 0;       // slots that received loads
-      uint32_t sf_used = 0;    // slots that received scale blocks
-      uint32_t full_par = 0;   // per slot: parity of its next full phase
-      uint32_t sf_par = 0;     // per slot: parity of its next full_sf phase
+      uint32_t used = 0;       // slots this thread loaded
+      uint32_t last_par = 0;   // per slot: parity of the last phase armed
+      uint32_t sf_used = 0;    // slots this thread loaded scales into
+      uint32_t sf_par = 0;     // per slot: parity of the next full_sf phase
       bool ok = true;
       for (int t = blockIdx.x; ok && t < p.tiles; t += gridDim.x) {
         int m0, n0;
         tile_coords(t, p.tiles_n, BN, m0, n0);
-        const int b0 = n0 / 128;  // first weight-scale block of the tile
-        const int nbl = min((n0 + BN - 1) / 128, nb_total - 1) - b0 + 1;
         for (int st = 0; st < nsteps; ++st, ++it) {
           const int s = it % kStages;
+          if (s % kProducers != warp) continue;
           const uint32_t ph = (it / kStages) & 1;
           if (!mbar_wait(&empty[s], ph ^ 1, p.wait, kErrTimeoutEmpty)) {
             ok = false;
@@ -191,13 +201,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (p.fault == 1 && it == 0) continue;  // test hook: this slot never fills
             const int nkb = min(4, kblocks - 4 * st);
             const uint32_t sfbytes = static_cast<uint32_t>(nkb) * 512;
-            mbar_arrive_expect_tx(&full_sf[s], sfbytes * (1 + nbl));
-            bulk_load(stage_sfa(s), p.sf_a + (static_cast<size_t>(m0 / 128) * kblocks + 4 * st) * 512,
+            const size_t koff = static_cast<size_t>(4 * st) * 512;
+            const uint8_t* wsf = p.sf_w + static_cast<size_t>(n0 / 128) * kblocks * 512 + koff;
+            mbar_arrive_expect_tx(&full_sf[s], sfbytes * (BN > 128 ? 3 : 2));
+            bulk_load(stage_sfa(s), p.sf_a + static_cast<size_t>(m0 / 128) * kblocks * 512 + koff,
                       sfbytes, &full_sf[s]);
-            for (int nb = 0; nb < nbl; ++nb)
-              bulk_load(stage_sfb(s) + nb * 2048,
-                        p.sf_w + (static_cast<size_t>(b0 + nb) * kblocks + 4 * st) * 512, sfbytes,
-                        &full_sf[s]);
+            bulk_load(stage_sfb(s), wsf, sfbytes, &full_sf[s]);
+            if (BN > 128) bulk_load(stage_sfb(s) + 2048, wsf + static_cast<size_t>(kblocks) * 512, sfbytes, &full_sf[s]);
             sf_used |= 1u << s;
             sf_par ^= 1u << s;
             mbar_arrive_expect_tx(&full[s], kATileBytes + L::kB);
@@ -213,19 +223,18 @@ __global__ void __launch_bounds__(kThreads, 1)
             tma_load_2d(stage_a(s), &tmap_lr, &full[s], 32 * j, m0);
           }
           used |= 1u << s;
-          full_par ^= 1u << s;
+          last_par = (last_par & ~(1u << s)) | (ph << s);
         }
       }
       // never leave the CTA with a copy still landing in its shared memory:
-      // every earlier phase of a slot completed before the slot was reused
+      // an earlier phase of a slot completed before the slot was armed again
       for (int s = 0; s < kStages; ++s) {
-        if (used & (1u << s))
-          mbar_wait(&full[s], ((full_par >> s) & 1u) ^ 1u, p.wait, kErrTimeoutDrain);
+        if (used & (1u << s)) mbar_wait(&full[s], (last_par >> s) & 1u, p.wait, kErrTimeoutDrain);
         if (sf_used & (1u << s))
           mbar_wait(&full_sf[s], ((sf_par >> s) & 1u) ^ 1u, p.wait, kErrTimeoutDrain);
       }
     }
-  } else if (warp == 1) {
+  } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ MMA ----
     if (lane == 0) {
       const uint32_t id_f16 = idesc_f16(128, BN, true);
@@ -234,8 +243,25 @@ __global__ void __launch_bounds__(kThreads, 1)
       // to the start-address field (shared addresses stay below 256 KB)
       const uint64_t da0 = make_sdesc(smem_u32(stage_a(0)), 16, 1024, kSwz128);
       const uint64_t db0 = make_sdesc(smem_u32(stage_b(0)), 16, 1024, kSwz128);
-      int it = 0, f = 0;                     // ring steps, FP4 steps
+      // Everything below is kept incremental (no divisions, unrolled MMAs):
+      // the tensor pipe holds about one MMA ahead of this thread, so scalar
+      // latency between MMAs is idle tensor time.
+      int s = 0;                             // ring slot of the next step
+      uint64_t soff = 0;                     // its descriptor offset (bytes >> 4)
+      int rg = 0;                            // scale region of the next FP4 step
+      uint32_t sfr = tmem + L::kSfCol;       // its first column
+      uint32_t sf_par = 0;                   // parity of each region's next sfready phase
       uint32_t lr_par = 0;                   // parity of each slot's next lrf phase
+      const int nkb_last = kblocks - 4 * (nk - 1);  // 64-K blocks of the last FP4 step
+      const int lr_k = p.r < 32 ? 1 : 2;     // low-rank k-steps per slice (hi and lo each)
+      auto advance = [&]() {
+        if (++s == kStages) {
+          s = 0;
+          soff = 0;
+        } else {
+          soff += L::kStage >> 4;
+        }
+      };
       int local = 0;                         // tiles done by this CTA
       bool ok = true;
       for (int t = blockIdx.x; ok && t < p.tiles; t += gridDim.x, ++local) {
@@ -248,103 +274,152 @@ __global__ void __launch_bounds__(kThreads, 1)
           break;
         }
         tc_fence_after();
-        for (int st = 0; st < nsteps; ++st, ++it) {
-          const int s = it % kStages;
-          const uint64_t soff = static_cast<uint64_t>((s * L::kStage) >> 4);
-          if (st < nk) {
-            const int rg = f & 1;
-            // the stagers arrive only after the slot's operands have landed
-            if (!mbar_wait(&sfready[rg], (f >> 1) & 1, p.wait, kErrTimeoutFull)) {
-              ok = false;
-              break;
-            }
-            tc_fence_after();
-            const uint32_t sfr = tmem + L::kSfCol + rg * kSfRegionCols;
-            const int nkb = min(4, kblocks - 4 * st);
-            for (int kk = 0; kk < nkb; ++kk)
-              umma_nvfp4(acc, da0 + soff + 2 * kk, db0 + soff + 2 * kk, id_fp4, sfr + 4 * kk,
-                         sfr + 16 + 8 * kk, (st > 0 || kk > 0) ? 1u : 0u);
-            umma_commit(&empty[s]);
-            umma_commit(&sffree[rg]);
-            ++f;
-          } else {
-            if (!mbar_wait(&lrf[s], (lr_par >> s) & 1u, p.wait, kErrTimeoutFull)) {
-              ok = false;
-              break;
-            }
-            lr_par ^= 1u << s;
-            tc_fence_after();
-            // A k-steps {0, 1} hold hi and {2, 3} lo of the slice's 32
-            // columns, both against B k-steps {0, 1} (r = 16: one of each)
-            const int ksteps = p.r < 32 ? 1 : 2;
-            for (int kk = 0; kk < ksteps; ++kk) {
-              umma_f16(acc, da0 + soff + 2 * kk, db0 + soff + 2 * kk, id_f16, 1u);
-              umma_f16(acc, da0 + soff + 2 * (2 + kk), db0 + soff + 2 * kk, id_f16, 1u);
-            }
-            umma_commit(&empty[s]);
+        for (int st = 0; st < nk; ++st) {
+          // the stagers arrive only after the slot's operands have landed
+          if (!mbar_wait(&sfready[rg], (sf_par >> rg) & 1u, p.wait, kErrTimeoutFull)) {
+            ok = false;
+            break;
           }
+          sf_par ^= 1u << rg;
+          tc_fence_after();
+          const uint64_t da = da0 + soff, db = db0 + soff;
+          if (st + 1 < nk || nkb_last == 4) {
+            umma_nvfp4(acc, da, db, id_fp4, sfr, sfr + 16, st > 0 ? 1u : 0u);
+#pragma unroll
+            for (int kk = 1; kk < 4; ++kk)
+              umma_nvfp4(acc, da + 2 * kk, db + 2 * kk, id_fp4, sfr + 4 * kk,
+                         sfr + 16 + L::kSfbCols * kk, 1u);
+          } else {
+            for (int kk = 0; kk < nkb_last; ++kk)
+              umma_nvfp4(acc, da + 2 * kk, db + 2 * kk, id_fp4, sfr + 4 * kk,
+                         sfr + 16 + L::kSfbCols * kk, (st > 0 || kk > 0) ? 1u : 0u);
+          }
+          umma_commit(&empty[s]);
+          umma_commit(&sffree[rg]);
+          if (++rg == L::kRegions) {
+            rg = 0;
+            sfr = tmem + L::kSfCol;
+          } else {
+            sfr += L::kSfRegionCols;
+          }
+          advance();
+        }
+        for (int j = 0; ok && j < nlr; ++j) {
+          if (!mbar_wait(&lrf[s], (lr_par >> s) & 1u, p.wait, kErrTimeoutFull)) {
+            ok = false;
+            break;
+          }
+          lr_par ^= 1u << s;
+          tc_fence_after();
+          // A k-steps {0, 1} hold hi and {2, 3} lo of the slice's 32
+          // columns, both against B k-steps {0, 1} (r = 16: one of each)
+          const uint64_t da = da0 + soff, db = db0 + soff;
+          for (int kk = 0; kk < lr_k; ++kk) {
+            umma_f16(acc, da + 2 * kk, db + 2 * kk, id_f16, 1u);
+            umma_f16(acc, da + 2 * (2 + kk), db + 2 * kk, id_f16, 1u);
+          }
+          umma_commit(&empty[s]);
+          advance();
         }
         if (ok) umma_commit(&acc_full[a]);
       }
     }
-  } else if (warp < 2 + kStagerWarps) {
+  } else if (warp < kMmaWarp + 1 + kStagerWarps) {  // stagers
     // ----------------------------------------------------------- stagers ----
     const int quad = warp & 3;               // TMEM lane quadrant this warp may access
     const int row = 32 * quad + lane;        // tile row of the low-rank A operand
     const uint32_t lane_off = static_cast<uint32_t>(32 * quad) << 16;
     const float gprod = __fmul_rn(*p.gs_a, *p.gs_w);
-    int it = 0, f = 0;
+    int ss = 0;                              // ring slot of the next step
+    uint32_t sph = 0;                        // its phase parity
     uint32_t sf_par = 0;                     // parity of each slot's next full_sf phase
+    int f = 0;                               // FP4 steps done
+    int rg = 0;                              // scale region of the next FP4 step
+    uint32_t free_par = 0;                   // parity of each region's next sffree phase
     bool ok = true;
+    // One FP4 step: the slot's scales into region rg.  Per 64-K block kk this
+    // lane needs line `lane` (16 bytes) of the activation block and the words
+    // of the weight blocks that hold tile rows 32j + lane: weight row n0 + 32j
+    // + lane sits in word ((n0 % 128 + 32j) % 128) / 32 of line `lane` of
+    // block (n0 + 32j) / 128.  BN = 128: the whole line of the one block.
+    // BN = 192, n0 % 128 == 0: the line of block 0 (rows 0-127), then words
+    // 0-1 of block 1 (rows 128-191); n0 % 128 == 64: words 2-3 of block 0
+    // (rows 0-63), then the line of block 1 (rows 64-191).
+    auto fp4_step = [&](bool hi64, int s, uint32_t ph) -> bool {
+      // region rg's previous user is FP4 step f - kRegions
+      if (f >= L::kRegions) {
+        if (!mbar_wait(&sffree[rg], (free_par >> rg) & 1u, p.wait, kErrTimeoutEmpty)) return false;
+        free_par ^= 1u << rg;
+      }
+      if (!mbar_wait(&full_sf[s], (sf_par >> s) & 1u, p.wait, kErrTimeoutFull)) return false;
+      sf_par ^= 1u << s;
+      tc_fence_after();
+      const uint8_t* sa = stage_sfa(s) + lane * 16;
+      const uint8_t* sb = stage_sfb(s) + lane * 16;
+      uint32_t va[16];
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk) {
+        const uint4 u = *reinterpret_cast<const uint4*>(sa + kk * 512);
+        va[4 * kk] = u.x;
+        va[4 * kk + 1] = u.y;
+        va[4 * kk + 2] = u.z;
+        va[4 * kk + 3] = u.w;
+      }
+      const uint32_t sfr = tmem + lane_off + L::kSfCol + rg * L::kSfRegionCols;
+      // SFA: column 4kk + j = bytes [4j, 4j + 4) of line `lane` of block kk
+      tmem_st_32x32b_x16(sfr, va);
+      // SFB: column 16 + (BN/32)kk + j holds tile row 32j + lane
+      if constexpr (BN == 128) {
+        uint32_t vb[16];
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+          const uint4 x = *reinterpret_cast<const uint4*>(sb + kk * 512);
+          vb[4 * kk] = x.x;
+          vb[4 * kk + 1] = x.y;
+          vb[4 * kk + 2] = x.z;
+          vb[4 * kk + 3] = x.w;
+        }
+        tmem_st_32x32b_x16(sfr + 16, vb);
+      } else {
+        uint32_t vb[24];
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+          const uint4 x = *reinterpret_cast<const uint4*>(sb + (hi64 ? 2048 : 0) + kk * 512);
+          const uint2 y = *reinterpret_cast<const uint2*>(sb + (hi64 ? 8 : 2048) + kk * 512);
+          const uint32_t lo[6] = {x.x, x.y, x.z, x.w, y.x, y.y};
+          const uint32_t hi[6] = {y.x, y.y, x.x, x.y, x.z, x.w};
+#pragma unroll
+          for (int j = 0; j < 6; ++j) vb[6 * kk + j] = hi64 ? hi[j] : lo[j];
+        }
+        const uint32_t v16[16] = {vb[0], vb[1], vb[2],  vb[3],  vb[4],  vb[5],  vb[6],  vb[7],
+                                  vb[8], vb[9], vb[10], vb[11], vb[12], vb[13], vb[14], vb[15]};
+        const uint32_t v8[8] = {vb[16], vb[17], vb[18], vb[19], vb[20], vb[21], vb[22], vb[23]};
+        tmem_st_32x32b_x16(sfr + 16, v16);
+        tmem_st_32x32b_x8(sfr + 32, v8);
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      // the MMA thread waits on sfready alone: make it imply the operands too
+      if (!mbar_wait(&full[s], ph, p.wait, kErrTimeoutFull)) return false;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sfready[rg]);
+      ++f;
+      rg = rg + 1 == L::kRegions ? 0 : rg + 1;
+      return true;
+    };
     for (int t = blockIdx.x; ok && t < p.tiles; t += gridDim.x) {
       int m0, n0;
       tile_coords(t, p.tiles_n, BN, m0, n0);
-      for (int st = 0; ok && st < nsteps; ++st, ++it) {
-        const int s = it % kStages;
-        const uint32_t ph = (it / kStages) & 1;
+      const bool hi64 = (n0 & 127) != 0;
+      for (int st = 0; ok && st < nsteps; ++st) {
+        const int s = ss;
+        const uint32_t ph = sph;
+        if (++ss == kStages) {  // the ring position of the next step
+          ss = 0;
+          sph ^= 1u;
+        }
         if (st < nk) {
-          // this FP4 step's scales into region rg (its previous user is FP4 step f - 2)
-          const int rg = f & 1;
-          if (f >= 2 && !mbar_wait(&sffree[rg], ((f >> 1) - 1) & 1, p.wait, kErrTimeoutEmpty)) {
-            ok = false;
-            break;
-          }
-          if (!mbar_wait(&full_sf[s], (sf_par >> s) & 1u, p.wait, kErrTimeoutFull)) {
-            ok = false;
-            break;
-          }
-          sf_par ^= 1u << s;
-          tc_fence_after();
-          const uint32_t sfr = tmem + lane_off + L::kSfCol + rg * kSfRegionCols;
-          const int nkb = min(4, kblocks - 4 * st);
-          const uint8_t* sfa = stage_sfa(s);
-          const uint8_t* sfb = stage_sfb(s);
-          for (int kk = 0; kk < nkb; ++kk) {
-            // SFA: column 4kk + j = bytes [4j, 4j + 4) of the block's line `lane`
-            const uint4 va = *reinterpret_cast<const uint4*>(sfa + kk * 512 + lane * 16);
-            tmem_st_32x32b_x4(sfr + 4 * kk, va.x, va.y, va.z, va.w);
-            // SFB: column 16 + 8kk + j holds tile row 32j + lane, which is
-            // weight row n0 + 32j + lane, in block (n0 + 32j + lane)/128 - n0/128
-            uint32_t vb[BN / 32];
-#pragma unroll
-            for (int j = 0; j < BN / 32; ++j) {
-              const int rr = (n0 & 127) + 32 * j;  // row offset from block n0/128
-              vb[j] = *reinterpret_cast<const uint32_t*>(sfb + (rr >> 7) * 2048 + kk * 512 +
-                                                         lane * 16 + ((rr & 127) >> 5) * 4);
-            }
-            tmem_st_32x32b_x4(sfr + 16 + 8 * kk, vb[0], vb[1], vb[2], vb[3]);
-            if constexpr (BN / 32 == 6) tmem_st_32x32b_x2(sfr + 20 + 8 * kk, vb[4], vb[5]);
-          }
-          tmem_st_wait();
-          tc_fence_before();
-          // the MMA thread waits on sfready alone: make it imply the operands too
-          if (!mbar_wait(&full[s], ph, p.wait, kErrTimeoutFull)) {
-            ok = false;
-            break;
-          }
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&sfready[rg]);
-          ++f;
+          ok = fp4_step(hi64, s, ph);
         } else {
           // the tile's low-rank A operand, in place over the slot's xl slice
           if (!mbar_wait(&full[s], ph, p.wait, kErrTimeoutFull)) {
@@ -388,72 +463,68 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // ---------------------------------------------------------- epilogue ----
-    const int ew = warp - 2 - kStagerWarps;  // 0..7
+    const int ew = warp - (kMmaWarp + 1 + kStagerWarps);  // 0..3
     const int quad = warp & 3;               // TMEM lane quadrant this warp may access
-    const int half = ew >> 2;                // which group of 64-column boxes
-    const int box0 = half == 0 ? 0 : L::kBoxes0;
-    const int nbox = half == 0 ? L::kBoxes0 : L::kBoxes - L::kBoxes0;
     const float alpha = __fdiv_rn(1.0f, __fmul_rn(*p.gs_a, *p.gs_w));
-    uint16_t* bsl = bias_s + ew * (L::kBoxes0 * 64);
+    uint16_t* bsl = bias_s + ew * BN;
     uint8_t* box = out_s + ew * L::kBoxBytes;
     uint8_t* brow = box + lane * 128;
-    int local = 0;
+    int local = 0;                           // tiles drained
     for (int t = blockIdx.x; t < p.tiles; t += gridDim.x, ++local) {
       int m0, n0;
       tile_coords(t, p.tiles_n, BN, m0, n0);
       const int a = local & 1;
-      // this warp's bias columns into its own shared-memory slice
-      for (int c = lane; c < nbox * 64; c += 32) {
-        const int col = n0 + 64 * box0 + c;
+      // the tile's bias columns into this warp's shared-memory copy
+      for (int c = lane; c < BN; c += 32) {
+        const int col = n0 + c;
         bsl[c] = (p.bias && col < p.N) ? p.bias[col] : static_cast<uint16_t>(0);
       }
       __syncwarp();
       if (!mbar_wait(&acc_full[a], (local >> 1) & 1, p.wait, kErrTimeoutAcc)) break;
       tc_fence_after();
-      // drain: α·acc + bias -> packed bf16
-      uint32_t packed[L::kBoxes0 * 32];
-      const uint32_t taddr = tmem + (static_cast<uint32_t>(32 * quad) << 16) + a * BN + 64 * box0;
+      const uint32_t taddr = tmem + (static_cast<uint32_t>(32 * quad) << 16) + a * BN;
+#pragma unroll 1
+      for (int j = 0; j < L::kBoxes; ++j) {
+        // α·acc + bias -> bf16 for columns [64j, 64j + 64) of this quadrant's rows
+        uint32_t packed[32];
 #pragma unroll
-      for (int c = 0; c < L::kBoxes0 * 4; c += 2) {  // 16-column chunks, two per load pair
-        if (c >= nbox * 4) break;
-        uint32_t v0[16], v1[16];
-        tmem_ld_32x32b_x16(taddr + c * 16, v0);
-        tmem_ld_32x32b_x16(taddr + (c + 1) * 16, v1);
-        tmem_ld_wait();
+        for (int c = 0; c < 4; c += 2) {  // 16-column chunks, two per load pair
+          uint32_t v0[16], v1[16];
+          tmem_ld_32x32b_x16(taddr + 64 * j + c * 16, v0);
+          tmem_ld_32x32b_x16(taddr + 64 * j + (c + 1) * 16, v1);
+          tmem_ld_wait();
 #pragma unroll
-        for (int u = 0; u < 2; ++u) {
-          const uint32_t* av = u ? v1 : v0;
-          const uint4* b4 = reinterpret_cast<const uint4*>(bsl + (c + u) * 16);
-          const uint4 bb0 = b4[0], bb1 = b4[1];
-          const uint32_t bw[8] = {bb0.x, bb0.y, bb0.z, bb0.w, bb1.x, bb1.y, bb1.z, bb1.w};
+          for (int u = 0; u < 2; ++u) {
+            const uint32_t* av = u ? v1 : v0;
+            const uint4* b4 = reinterpret_cast<const uint4*>(bsl + 64 * j + (c + u) * 16);
+            const uint4 bb0 = b4[0], bb1 = b4[1];
+            const uint32_t bw[8] = {bb0.x, bb0.y, bb0.z, bb0.w, bb1.x, bb1.y, bb1.z, bb1.w};
 #pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            const float lo = __fadd_rn(__fmul_rn(__uint_as_float(av[2 * e]), alpha),
-                                       __uint_as_float(bw[e] << 16));
-            const float hi = __fadd_rn(__fmul_rn(__uint_as_float(av[2 * e + 1]), alpha),
-                                       __uint_as_float(bw[e] & 0xFFFF0000u));
-            packed[(c + u) * 8 + e] = pack_bf16x2(lo, hi);
+            for (int e = 0; e < 8; ++e) {
+              const float lo = __fadd_rn(__fmul_rn(__uint_as_float(av[2 * e]), alpha),
+                                         __uint_as_float(bw[e] << 16));
+              const float hi = __fadd_rn(__fmul_rn(__uint_as_float(av[2 * e + 1]), alpha),
+                                         __uint_as_float(bw[e] & 0xFFFF0000u));
+              packed[(c + u) * 8 + e] = pack_bf16x2(lo, hi);
+            }
           }
         }
-      }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&acc_empty[a]);  // the MMAs may refill this accumulator
-      // store: one 32 x 64 staging box per 64 columns, 128-byte swizzle
-#pragma unroll
-      for (int j = 0; j < L::kBoxes0; ++j) {
-        if (j >= nbox) break;
-        if (lane == 0) bulk_wait_group_read<0>();  // the previous box has left shared memory
+        if (j == L::kBoxes - 1) {  // the accumulator is drained: the MMAs may refill it
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&acc_empty[a]);
+        }
+        // 32 x 64 staging box, 128-byte swizzle
+        if (lane == 0) bulk_wait_group_read<0>();  // the previous store has read the box
         __syncwarp();
 #pragma unroll
         for (int q = 0; q < 8; ++q)
           *reinterpret_cast<uint4*>(brow + ((q ^ (lane & 7)) << 4)) =
-              make_uint4(packed[32 * j + 4 * q], packed[32 * j + 4 * q + 1],
-                         packed[32 * j + 4 * q + 2], packed[32 * j + 4 * q + 3]);
+              make_uint4(packed[4 * q], packed[4 * q + 1], packed[4 * q + 2], packed[4 * q + 3]);
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) {
-          tma_store_2d(&tmap_y, box, n0 + 64 * (box0 + j), m0 + 32 * quad);
+          tma_store_2d(&tmap_y, box, n0 + 64 * j, m0 + 32 * quad);
           bulk_commit_group();
         }
       }
@@ -462,7 +533,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 1) {
+  if (warp == kMmaWarp) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
@@ -474,7 +545,7 @@ svdq_status launch_bn(const LaunchCtx& ctx, const CUtensorMap& ta, const CUtenso
                       GemmParams p) {
   using L = Layout<BN>;
   const size_t smem = 1024 + static_cast<size_t>(L::kRing) + kEpiWarps * L::kBoxBytes + L::kBias +
-                      8 * (4 * kStages + 8) + 16;
+                      8 * (4 * kStages + 2 * kMaxRegions + 4) + 16;
   static bool attr_done[64] = {};
   if (!attr_done[ctx.device & 63]) {
     cudaFuncSetAttribute(w4a4_gemm_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,

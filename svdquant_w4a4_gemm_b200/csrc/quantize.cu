@@ -12,8 +12,10 @@
 // (one persistent CTA per SM), so the memory pipeline never drains between
 // work items and the load is balanced to one sub-tile.
 //   warp 0       TMA producer: x sub-tiles and the matching 64-column slices
-//                of L1ᵀ into a kStages-deep shared-memory ring.  The first
-//                kStages loads are issued before the CTA-wide set-up, while
+//                of L1ᵀ into a shared-memory ring as deep as shared memory
+//                allows (up to 8 sub-tiles: the loads come from HBM, and the
+//                ring must cover its latency).  The first loads of the ring
+//                are issued before the CTA-wide set-up, while
 //                the other warps compute RN(1/s) once for every column this
 //                CTA's range touches.
 //   warp 1       TMEM owner; one thread issues the down-projection as
@@ -46,7 +48,7 @@ namespace {
 
 constexpr int kBM = 128;
 constexpr int kSubK = 64;
-constexpr int kStages = 4;
+constexpr int kMaxStages = 8;
 constexpr int kQuantWarps = 16;
 constexpr int kEpiWarps = 4;
 constexpr int kThreads = 32 * (2 + kQuantWarps + kEpiWarps);
@@ -55,6 +57,7 @@ constexpr uint32_t kXTileBytes = kBM * kSubK * 2;
 struct QuantParams {
   int M, K, r;
   int units;              // ceil(M/128) * (K/64) sub-tiles
+  int stages;             // ring depth, <= kMaxStages
   const float* smooth_s;  // [K] or null
   const float* gs_in;     // static tensor scale, or null for dynamic
   const float* amax_src;  // dynamic: amax bits (written by the amax pass)
@@ -91,13 +94,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                                              ~static_cast<uintptr_t>(1023));
   const uint32_t l1_bytes = static_cast<uint32_t>(p.r) * 128u;
   uint8_t* xs = base;
-  uint8_t* ls = xs + kStages * kXTileBytes;
-  float* inv_s = reinterpret_cast<float*>(ls + kStages * l1_bytes);   // [K], touched columns
+  const int ns = p.stages;
+  uint8_t* ls = xs + ns * kXTileBytes;
+  float* inv_s = reinterpret_cast<float*>(ls + ns * l1_bytes);        // [K], touched columns
   float* gs_over_d = inv_s + p.K;                                     // [128] by E4M3 code
   uint64_t* full = reinterpret_cast<uint64_t*>(gs_over_d + 128);
-  uint64_t* qdone = full + kStages;
-  uint64_t* empty = qdone + kStages;
-  uint64_t* acc_full = empty + kStages;  // [2]
+  uint64_t* qdone = full + kMaxStages;
+  uint64_t* empty = qdone + kMaxStages;
+  uint64_t* acc_full = empty + kMaxStages;  // [2]
   uint64_t* acc_empty = acc_full + 2;    // [2]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
 
@@ -108,11 +112,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   int u0, u1;
   unit_range(p.units, u0, u1);
 
-  // Warp 0 sets up the barriers and issues the first kStages loads right
+  // Warp 0 sets up the barriers and issues the first ns loads right
   // away; the rest of the CTA fills the RN(1/s) and RN(gs/scale) tables in
   // the meantime.  Nobody else touches a barrier before the __syncthreads.
   if (warp == 0 && lane == 0) {
-    for (int s = 0; s < kStages; ++s) {
+    for (int s = 0; s < ns; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&qdone[s], kQuantWarps);
       mbar_init(&empty[s], has_lr ? 1 : kQuantWarps);
@@ -124,7 +128,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     fence_mbar_init();
     tma_prefetch_desc(&tmap_x);
     if (has_lr) tma_prefetch_desc(&tmap_l1);
-    for (int u = u0; u < min(u1, u0 + kStages); ++u) {
+    for (int u = u0; u < min(u1, u0 + ns); ++u) {
       const int s = u - u0;
       const int rb = u / kblocks, kb = u % kblocks;
       mbar_arrive_expect_tx(&full[s], kXTileBytes + (has_lr ? l1_bytes : 0u));
@@ -164,11 +168,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0) {
     // ------------------------------------------------------- producer ----
     if (lane == 0) {
-      int issued = min(u1 - u0, kStages);  // issued before the set-up sync
-      for (int u = u0 + kStages; u < u1; ++u) {
+      int issued = min(u1 - u0, ns);  // issued before the set-up sync
+      for (int u = u0 + ns; u < u1; ++u) {
         const int i = u - u0;
-        const int s = i % kStages;
-        const uint32_t ph = (i / kStages) & 1;
+        const int s = i % ns;
+        const uint32_t ph = (i / ns) & 1;
         if (!mbar_wait(&empty[s], ph ^ 1, p.wait, kErrTimeoutEmpty)) break;
         const int rb = u / kblocks, kb = u % kblocks;
         mbar_arrive_expect_tx(&full[s], kXTileBytes + (has_lr ? l1_bytes : 0u));
@@ -177,8 +181,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         issued = i + 1;
       }
       // never leave the CTA with a copy still landing in its shared memory
-      for (int i = max(0, issued - kStages); i < issued; ++i)
-        mbar_wait(&full[i % kStages], (i / kStages) & 1, p.wait, kErrTimeoutDrain);
+      for (int i = max(0, issued - ns); i < issued; ++i)
+        mbar_wait(&full[i % ns], (i / ns) & 1, p.wait, kErrTimeoutDrain);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA ----
@@ -188,8 +192,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool first = true;       // first sub-tile of the current segment
       for (int u = u0; u < u1; ++u) {
         const int i = u - u0;
-        const int s = i % kStages;
-        const uint32_t ph = (i / kStages) & 1;
+        const int s = i % ns;
+        const uint32_t ph = (i / ns) & 1;
         const int buf = seg & 1;
         if (first && seg >= 2 &&
             !mbar_wait(&acc_empty[buf], ((seg >> 1) - 1) & 1, p.wait, kErrTimeoutAcc))
@@ -224,8 +228,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const size_t kbytes = static_cast<size_t>(p.K) / 2;
     for (int u = u0; u < u1; ++u) {
       const int i = u - u0;
-      const int s = i % kStages;
-      const uint32_t ph = (i / kStages) & 1;
+      const int s = i % ns;
+      const uint32_t ph = (i / ns) & 1;
       if (!mbar_wait(&full[s], ph, p.wait, kErrTimeoutFull)) break;
       const int rb = u / kblocks, kb = u % kblocks;
       const int grow = rb * kBM + row;
@@ -364,9 +368,23 @@ __global__ void act_scale_finalize_kernel(float* gs) {
 
 }  // namespace
 
+namespace {
+constexpr size_t kSmemLimit = 227 * 1024;
+size_t quantize_fixed_bytes(int64_t K) {
+  return 1024 + static_cast<size_t>(K) * 4 + 128 * 4 + 8 * (3 * kMaxStages + 4) + 16;
+}
+// Ring depth: as many sub-tiles as fit next to the RN(1/s) table, 2..8.
+int quantize_stages(int64_t K, int r) {
+  const size_t fixed = quantize_fixed_bytes(K);
+  const size_t per = kXTileBytes + static_cast<size_t>(r) * 128;
+  const int fit = fixed < kSmemLimit ? static_cast<int>((kSmemLimit - fixed) / per) : 0;
+  return std::max(2, std::min(kMaxStages, fit));
+}
+}  // namespace
+
 size_t quantize_smem_bytes(int64_t K, int r) {
-  return 1024 + kStages * (kXTileBytes + static_cast<size_t>(r) * 128) + static_cast<size_t>(K) * 4 +
-         128 * 4 + 8 * (3 * kStages + 4) + 16;
+  return quantize_fixed_bytes(K) +
+         static_cast<size_t>(quantize_stages(K, r)) * (kXTileBytes + static_cast<size_t>(r) * 128);
 }
 
 svdq_status launch_quantize_act(const LaunchCtx& ctx, const void* x, int64_t M, int64_t K,
@@ -386,6 +404,7 @@ svdq_status launch_quantize_act(const LaunchCtx& ctx, const void* x, int64_t M, 
   p.K = static_cast<int>(K);
   p.r = r;
   p.units = static_cast<int>(((M + kBM - 1) / kBM) * (K / kSubK));
+  p.stages = quantize_stages(K, r);
   p.smooth_s = smooth_s;
   p.gs_in = act_gscale;
   p.amax_src = act_gscale ? nullptr : act_gscale_out;
