@@ -274,34 +274,35 @@ __global__ void __launch_bounds__(kThreads, 1)
           break;
         }
         tc_fence_after();
+        bool ready = false;                  // the next step's sfready phase is known complete
         for (int st = 0; st < nk; ++st) {
           // the stagers arrive only after the slot's operands have landed
-          if (!mbar_wait(&sfready[rg], (sf_par >> rg) & 1u, p.wait, kErrTimeoutFull)) {
+          if (!ready && !mbar_wait(&sfready[rg], (sf_par >> rg) & 1u, p.wait, kErrTimeoutFull)) {
             ok = false;
             break;
           }
           sf_par ^= 1u << rg;
           tc_fence_after();
           const uint64_t da = da0 + soff, db = db0 + soff;
+          const int rg_next = rg + 1 == L::kRegions ? 0 : rg + 1;
           if (st + 1 < nk || nkb_last == 4) {
             umma_nvfp4(acc, da, db, id_fp4, sfr, sfr + 16, st > 0 ? 1u : 0u);
-#pragma unroll
-            for (int kk = 1; kk < 4; ++kk)
-              umma_nvfp4(acc, da + 2 * kk, db + 2 * kk, id_fp4, sfr + 4 * kk,
-                         sfr + 16 + L::kSfbCols * kk, 1u);
+            umma_nvfp4(acc, da + 2, db + 2, id_fp4, sfr + 4, sfr + 16 + L::kSfbCols, 1u);
+            umma_nvfp4(acc, da + 4, db + 4, id_fp4, sfr + 8, sfr + 16 + 2 * L::kSfbCols, 1u);
+            // look at the next step's barrier while the tensor pipe is busy:
+            // waiting for it after the last MMA would leave the pipe idle
+            ready = st + 1 < nk && mbar_test(&sfready[rg_next], (sf_par >> rg_next) & 1u);
+            umma_nvfp4(acc, da + 6, db + 6, id_fp4, sfr + 12, sfr + 16 + 3 * L::kSfbCols, 1u);
           } else {
+            ready = false;
             for (int kk = 0; kk < nkb_last; ++kk)
               umma_nvfp4(acc, da + 2 * kk, db + 2 * kk, id_fp4, sfr + 4 * kk,
                          sfr + 16 + L::kSfbCols * kk, (st > 0 || kk > 0) ? 1u : 0u);
           }
           umma_commit(&empty[s]);
           umma_commit(&sffree[rg]);
-          if (++rg == L::kRegions) {
-            rg = 0;
-            sfr = tmem + L::kSfCol;
-          } else {
-            sfr += L::kSfRegionCols;
-          }
+          rg = rg_next;
+          sfr = rg == 0 ? tmem + L::kSfCol : sfr + L::kSfRegionCols;
           advance();
         }
         for (int j = 0; ok && j < nlr; ++j) {
