@@ -200,27 +200,28 @@ def bench_device(args, rank, world, dev):
     sv.check_device_errors()
 
     # ---- the K timed steps, captured once into a CUDA graph so that the
-    # device time is not limited by host launch overhead; external timing
-    # events between the two kernels of every step give per-kernel times ----
+    # device time is not limited by host launch overhead ----
     gsteps = min(args.steps, 200)                 # steps per captured graph
     replays = max(1, -(-args.steps // gsteps))
-    ev = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(3)]
-          for _ in range(gsteps)]
-    graph = torch.cuda.CUDAGraph()
     cap = torch.cuda.Stream(dev)
-    cap.wait_stream(stream)
-    with torch.cuda.graph(graph, stream=cap):
-        for i in range(gsteps):
-            s = sets[i % nsets]
-            e0, e1, e2 = ev[i]
-            e0.record()
-            sv.quantize_act(s["x"], s["w"].smooth, s["w"].L1t, s["gs"],
-                            out=(s["q"], s["sf"], s["lora"], s["gso"]))
-            e1.record()
-            sv.w4a4_linear(s["q"], s["sf"], s["gso"], s["lora"], s["w"], y=s["y"])
-            e2.record()
-    graph.replay()                      # untimed: uploads the graph
-    torch.cuda.synchronize(dev)
+
+    def capture(body):
+        g = torch.cuda.CUDAGraph()
+        cap.wait_stream(stream)
+        with torch.cuda.graph(g, stream=cap):
+            for i in range(gsteps):
+                body(sets[i % nsets])
+        g.replay()                      # untimed: uploads the graph
+        torch.cuda.synchronize(dev)
+        return g
+
+    def k1(s):
+        sv.quantize_act(s["x"], s["w"].smooth, s["w"].L1t, s["gs"], out=(s["q"], s["sf"], s["lora"], s["gso"]))
+
+    def k2(s):
+        sv.w4a4_linear(s["q"], s["sf"], s["gso"], s["lora"], s["w"], y=s["y"])
+
+    graph = capture(lambda s: (k1(s), k2(s)))
     sv.check_device_errors()
 
     if world > 1:
@@ -240,8 +241,22 @@ def bench_device(args, rank, world, dev):
     steps_done = gsteps * replays
     total_ms, _ = aggregate(t_start.elapsed_time(t_end), steps_done,
                             layer_flops(CASE.M, CASE.K, CASE.N, CASE.r), world, dev)
-    k1_us = [e[0].elapsed_time(e[1]) * 1e3 for e in ev]
-    k2_us = [e[1].elapsed_time(e[2]) * 1e3 for e in ev]
+    # ---- per-kernel device times: each kernel alone, in a graph of its own
+    # over the same rotating sets (events around whole replays, on the stream
+    # the kernels run on) ----
+    per_kernel = {}
+    for name, body in (("k1", k1), ("k2", k2)):
+        g = capture(body)
+        reps = max(1, min(replays, 10))
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(reps):
+            g.replay()
+        b.record(stream)
+        torch.cuda.synchronize(dev)
+        per_kernel[name] = [a.elapsed_time(b) * 1e3 / (reps * gsteps)]
+        del g
+    k1_us, k2_us = per_kernel["k1"], per_kernel["k2"]
 
     # ---- e2e: the same call with host buffers, copies inside the timed region ----
     x_host = sets[0]["x"].cpu().pin_memory()

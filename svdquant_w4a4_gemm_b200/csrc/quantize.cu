@@ -13,7 +13,7 @@
 // work items and the load is balanced to one sub-tile.
 //   warp 0       TMA producer: x sub-tiles and the matching 64-column slices
 //                of L1ᵀ into a shared-memory ring as deep as shared memory
-//                allows (up to 8 sub-tiles: the loads come from HBM, and the
+//                allows (up to 12 sub-tiles: the loads come from HBM, and the
 //                ring must cover its latency).  The first loads of the ring
 //                are issued before the CTA-wide set-up, while
 //                the other warps compute RN(1/s) once for every column this
@@ -23,16 +23,17 @@
 //                the quantized tile's bf16(x̂) and the L1ᵀ slice into a TMEM
 //                accumulator; a new accumulator (of two) per run of
 //                sub-tiles in the same 128-row block ("segment").
-//   warps 2-17   quantizers: one thread = one row x one 16-element group
-//                (a warp = 8 rows x the tile's 4 groups, so four consecutive
-//                lanes write 32 contiguous code bytes and the row's 4 scale
-//                bytes): x̂ = x·inv_s, group max, E4M3 scale
+//   warps 2-9    quantizers, one sub-tile per warp (so up to 8 sub-tiles are
+//                worked on at once; with all warps on one sub-tile, each
+//                sub-tile costs a full dependent chain of latencies): lane l
+//                takes rows l, l+32, l+64, l+96 and each row's four 16-element
+//                groups: x̂ = x·inv_s, group max, E4M3 scale
 //                (cvt.rn.satfinite.e4m3x2; RN(gs / scale) from a per-CTA
 //                table of the 127 scale codes), E2M1 codes (cvt.rn.satfinite
-//                .e2m1x2), an 8-byte code store, a 1-byte scale store into
-//                the 128x4 block layout, and bf16(x̂) written back over the
-//                tile for the MMA.
-//   warps 18-21  epilogue: when a segment's accumulator is complete, TMEM ->
+//                .e2m1x2), the row's 32 code bytes and 4 scale bytes (one
+//                word in the 128x4 block layout), and bf16(x̂) written back
+//                over the tile for the MMA.
+//   warps 10-13  epilogue: when a segment's accumulator is complete, TMEM ->
 //                registers -> float4 atomics into xl (zeroed beforehand:
 //                a row block's K range can span several CTAs), then release
 //                the accumulator.
@@ -48,8 +49,8 @@ namespace {
 
 constexpr int kBM = 128;
 constexpr int kSubK = 64;
-constexpr int kMaxStages = 8;
-constexpr int kQuantWarps = 16;
+constexpr int kMaxStages = 12;
+constexpr int kQuantWarps = 8;   // one sub-tile each, so up to 8 in flight
 constexpr int kEpiWarps = 4;
 constexpr int kThreads = 32 * (2 + kQuantWarps + kEpiWarps);
 constexpr uint32_t kXTileBytes = kBM * kSubK * 2;
@@ -118,8 +119,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0 && lane == 0) {
     for (int s = 0; s < ns; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&qdone[s], kQuantWarps);
-      mbar_init(&empty[s], has_lr ? 1 : kQuantWarps);
+      mbar_init(&qdone[s], 1);
+      mbar_init(&empty[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&acc_full[b], 1);
@@ -188,30 +189,37 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------ MMA ----
     if (has_lr && lane == 0) {
       const uint32_t idesc = idesc_f16(128, static_cast<uint32_t>(p.r), true);
+      // descriptors of slot 0; a slot adds its byte offset >> 4 (shared
+      // addresses stay below 256 KB).  No divisions in this loop: the tensor
+      // pipe idles while the issuing thread computes.
+      const uint64_t da0 = make_sdesc(smem_u32(xs), 16, 1024, kSwz128);
+      const uint64_t db0 = make_sdesc(smem_u32(ls), 16, 1024, kSwz128);
       int seg = 0;             // segments started by this CTA
       bool first = true;       // first sub-tile of the current segment
+      int s = 0;               // ring slot of unit u
+      uint32_t ph = 0;         // its phase parity
+      int kb = u0 % kblocks;   // 64-column block of unit u
       for (int u = u0; u < u1; ++u) {
-        const int i = u - u0;
-        const int s = i % ns;
-        const uint32_t ph = (i / ns) & 1;
         const int buf = seg & 1;
         if (first && seg >= 2 &&
             !mbar_wait(&acc_empty[buf], ((seg >> 1) - 1) & 1, p.wait, kErrTimeoutAcc))
           break;
         if (!mbar_wait(&qdone[s], ph, p.wait, kErrTimeoutFull)) break;
         tc_fence_after();
-        const uint32_t a0 = smem_u32(xs + s * kXTileBytes);
-        const uint32_t b0 = smem_u32(ls + s * l1_bytes);
+        const uint64_t da = da0 + ((static_cast<uint32_t>(s) * kXTileBytes) >> 4);
+        const uint64_t db = db0 + ((static_cast<uint32_t>(s) * l1_bytes) >> 4);
         const uint32_t d = tmem + buf * static_cast<uint32_t>(p.r);
+        umma_f16(d, da, db, idesc, first ? 0u : 1u);
 #pragma unroll
-        for (int kk = 0; kk < kSubK / 16; ++kk) {
-          const uint64_t ad = make_sdesc(a0 + kk * 32, 16, 1024, kSwz128);
-          const uint64_t bd = make_sdesc(b0 + kk * 32, 16, 1024, kSwz128);
-          umma_f16(d, ad, bd, idesc, (!first || kk > 0) ? 1u : 0u);
-        }
+        for (int kk = 1; kk < kSubK / 16; ++kk) umma_f16(d, da + 2 * kk, db + 2 * kk, idesc, 1u);
         umma_commit(&empty[s]);
         first = false;
-        const bool seg_end = (u + 1 == u1) || ((u + 1) / kblocks != u / kblocks);
+        if (++s == ns) {
+          s = 0;
+          ph ^= 1u;
+        }
+        const bool seg_end = (u + 1 == u1) || (kb + 1 == kblocks);  // the row block ends
+        kb = kb + 1 == kblocks ? 0 : kb + 1;
         if (seg_end) {
           umma_commit(&acc_full[buf]);
           ++seg;
@@ -222,63 +230,79 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp < 2 + kQuantWarps) {
     // ------------------------------------------------------ quantizers ----
     const int qw = warp - 2;
-    const int row = 8 * qw + (lane >> 2);  // row within the tile
-    const int g = lane & 3;                // which 16-element group of the 64 columns
+    // Each warp quantizes whole sub-tiles (units i = qw, qw + 8, ...), so up
+    // to 8 sub-tiles are in flight at once and each lane has 16 independent
+    // groups to interleave: lane l takes rows l, l + 32, l + 64, l + 96 of
+    // the tile, each row's four 16-element groups.
     if (p.gs_copy && blockIdx.x == 0 && threadIdx.x == 64) *p.gs_copy = gs;
     const size_t kbytes = static_cast<size_t>(p.K) / 2;
-    for (int u = u0; u < u1; ++u) {
+    for (int u = u0 + qw; u < u1; u += kQuantWarps) {
       const int i = u - u0;
       const int s = i % ns;
       const uint32_t ph = (i / ns) & 1;
       if (!mbar_wait(&full[s], ph, p.wait, kErrTimeoutFull)) break;
       const int rb = u / kblocks, kb = u % kblocks;
-      const int grow = rb * kBM + row;
-      uint8_t* trow = xs + s * kXTileBytes + row * 128;
-      const int kc0 = kb * kSubK + 16 * g;  // first column of this thread's group
-      uint8_t* c0p = trow + (((2 * g) ^ (row & 7)) << 4);
-      uint8_t* c1p = trow + (((2 * g + 1) ^ (row & 7)) << 4);
-      const uint4 v0 = *reinterpret_cast<const uint4*>(c0p);
-      const uint4 v1 = *reinterpret_cast<const uint4*>(c1p);
-      const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
-      float xh[16];
-      const float4* is4 = reinterpret_cast<const float4*>(inv_s + kc0);
+      const float* isk = inv_s + kb * kSubK;
+      uint8_t* sfb = p.sf_out + (static_cast<size_t>(rb) * kblocks + kb) * 512 + lane * 16;
+#pragma unroll 1
+      for (int j = 0; j < 4; ++j) {
+        const int row = lane + 32 * j;
+        const int grow = rb * kBM + row;
+        uint8_t* trow = xs + s * kXTileBytes + row * 128;
+        uint32_t codes[8];
+        uint32_t sfw = 0;  // the row's four scale bytes
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const float4 iv = is4[q];
-        xh[4 * q + 0] = __fmul_rn(bf16lo(w[2 * q]), iv.x);
-        xh[4 * q + 1] = __fmul_rn(bf16hi(w[2 * q]), iv.y);
-        xh[4 * q + 2] = __fmul_rn(bf16lo(w[2 * q + 1]), iv.z);
-        xh[4 * q + 3] = __fmul_rn(bf16hi(w[2 * q + 1]), iv.w);
+        for (int g = 0; g < 4; ++g) {
+          uint8_t* c0p = trow + (((2 * g) ^ (row & 7)) << 4);
+          uint8_t* c1p = trow + (((2 * g + 1) ^ (row & 7)) << 4);
+          const uint4 v0 = *reinterpret_cast<const uint4*>(c0p);
+          const uint4 v1 = *reinterpret_cast<const uint4*>(c1p);
+          const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+          float xh[16];
+          const float4* is4 = reinterpret_cast<const float4*>(isk + 16 * g);
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const float4 iv = is4[q];
+            xh[4 * q + 0] = __fmul_rn(bf16lo(w[2 * q]), iv.x);
+            xh[4 * q + 1] = __fmul_rn(bf16hi(w[2 * q]), iv.y);
+            xh[4 * q + 2] = __fmul_rn(bf16lo(w[2 * q + 1]), iv.z);
+            xh[4 * q + 3] = __fmul_rn(bf16hi(w[2 * q + 1]), iv.w);
+          }
+          float amax = 0.0f;
+#pragma unroll
+          for (int e = 0; e < 16; ++e) amax = fmaxf(amax, fabsf(xh[e]));
+          const float t = __fmul_rn(__fdiv_rn(amax, 6.0f), gs);
+          const uint32_t sf = cvt_e4m3(t);
+          const float inv = gs_over_d[sf & 127u];  // RN(gs / dec(sf)); 0 for a zero scale
+          sfw |= sf << (8 * g);
+          // cvt.rn.satfinite.e2m1x2 rounds ties to even and keeps the sign of
+          // a value that rounds to zero (code 0x8), as the format requires;
+          // the bit-exact tests hold it to that
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            float q8[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) q8[e] = __fmul_rn(xh[8 * h + e], inv);
+            codes[2 * g + h] = cvt_e2m1x8(q8);
+          }
+          if (has_lr) {  // bf16(x̂) back over the tile, for the down-projection
+            *reinterpret_cast<uint4*>(c0p) = make_uint4(pack_bf16x2(xh[0], xh[1]), pack_bf16x2(xh[2], xh[3]),
+                                                        pack_bf16x2(xh[4], xh[5]), pack_bf16x2(xh[6], xh[7]));
+            *reinterpret_cast<uint4*>(c1p) = make_uint4(pack_bf16x2(xh[8], xh[9]), pack_bf16x2(xh[10], xh[11]),
+                                                        pack_bf16x2(xh[12], xh[13]), pack_bf16x2(xh[14], xh[15]));
+          }
+        }
+        if (grow < p.M) {  // the row's 32 code bytes of this 64-column block
+          uint4* dst = reinterpret_cast<uint4*>(p.q_out + static_cast<size_t>(grow) * kbytes + kb * (kSubK / 2));
+          dst[0] = make_uint4(codes[0], codes[1], codes[2], codes[3]);
+          dst[1] = make_uint4(codes[4], codes[5], codes[6], codes[7]);
+        }
+        // the row's four scales: bytes (row % 32)·16 + (row / 32)·4 + g of the
+        // 512-byte block; rows past M inside the last 128-row block hold
+        // zero-filled x, so their scales are the zero padding the layout needs
+        *reinterpret_cast<uint32_t*>(sfb + 4 * j) = sfw;
       }
-      float amax = 0.0f;
-#pragma unroll
-      for (int e = 0; e < 16; ++e) amax = fmaxf(amax, fabsf(xh[e]));
-      const float t = __fmul_rn(__fdiv_rn(amax, 6.0f), gs);
-      const uint32_t sf = cvt_e4m3(t);
-      const float inv = gs_over_d[sf & 127u];  // RN(gs / dec(sf)); 0 for a zero scale
-      // cvt.rn.satfinite.e2m1x2 rounds ties to even and keeps the sign of a
-      // value that rounds to zero (code 0x8), as the format requires; the
-      // bit-exact tests hold it to that
-      uint32_t codes[2];
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        float q8[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) q8[e] = __fmul_rn(xh[8 * h + e], inv);
-        codes[h] = cvt_e2m1x8(q8);
-      }
-      if (grow < p.M)
-        *reinterpret_cast<uint2*>(p.q_out + static_cast<size_t>(grow) * kbytes + kc0 / 2) =
-            make_uint2(codes[0], codes[1]);
-      // rows past M inside the last 128-row block hold zero-filled x, so
-      // their scales are written as the zero padding the layout requires
-      p.sf_out[(static_cast<size_t>(rb) * kblocks + kb) * 512 + (row & 31) * 16 + (row >> 5) * 4 + g] =
-          static_cast<uint8_t>(sf);
       if (has_lr) {
-        *reinterpret_cast<uint4*>(c0p) = make_uint4(pack_bf16x2(xh[0], xh[1]), pack_bf16x2(xh[2], xh[3]),
-                                                    pack_bf16x2(xh[4], xh[5]), pack_bf16x2(xh[6], xh[7]));
-        *reinterpret_cast<uint4*>(c1p) = make_uint4(pack_bf16x2(xh[8], xh[9]), pack_bf16x2(xh[10], xh[11]),
-                                                    pack_bf16x2(xh[12], xh[13]), pack_bf16x2(xh[14], xh[15]));
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) mbar_arrive(&qdone[s]);
@@ -373,7 +397,7 @@ constexpr size_t kSmemLimit = 227 * 1024;
 size_t quantize_fixed_bytes(int64_t K) {
   return 1024 + static_cast<size_t>(K) * 4 + 128 * 4 + 8 * (3 * kMaxStages + 4) + 16;
 }
-// Ring depth: as many sub-tiles as fit next to the RN(1/s) table, 2..8.
+// Ring depth: as many sub-tiles as fit next to the RN(1/s) table, 2..12.
 int quantize_stages(int64_t K, int r) {
   const size_t fixed = quantize_fixed_bytes(K);
   const size_t per = kXTileBytes + static_cast<size_t>(r) * 128;
