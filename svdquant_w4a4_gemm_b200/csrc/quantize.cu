@@ -244,7 +244,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int rb = u / kblocks, kb = u % kblocks;
       const float* isk = inv_s + kb * kSubK;
       uint8_t* sfb = p.sf_out + (static_cast<size_t>(rb) * kblocks + kb) * 512 + lane * 16;
-#pragma unroll 1
+#pragma unroll 2
       for (int j = 0; j < 4; ++j) {
         const int row = lane + 32 * j;
         const int grow = rb * kBM + row;
@@ -268,9 +268,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             xh[4 * q + 2] = __fmul_rn(bf16lo(w[2 * q + 1]), iv.z);
             xh[4 * q + 3] = __fmul_rn(bf16hi(w[2 * q + 1]), iv.w);
           }
-          float amax = 0.0f;
+          // group max as a tree (max is exact, so the order does not matter)
+          float m8[8];
 #pragma unroll
-          for (int e = 0; e < 16; ++e) amax = fmaxf(amax, fabsf(xh[e]));
+          for (int e = 0; e < 8; ++e) m8[e] = fmaxf(fabsf(xh[e]), fabsf(xh[e + 8]));
+#pragma unroll
+          for (int e = 0; e < 4; ++e) m8[e] = fmaxf(m8[e], m8[e + 4]);
+          const float amax = fmaxf(fmaxf(m8[0], m8[2]), fmaxf(m8[1], m8[3]));
           const float t = __fmul_rn(__fdiv_rn(amax, 6.0f), gs);
           const uint32_t sf = cvt_e4m3(t);
           const float inv = gs_over_d[sf & 127u];  // RN(gs / dec(sf)); 0 for a zero scale
