@@ -126,20 +126,21 @@ class ClockSampler:
 
 
 # ------------------------------------------------------- device workload --
-def make_sets(dev, l2_bytes):
+def make_sets(dev, l2_bytes, case=None):
     """Independent copies of one layer (weights + activations + outputs),
     prepared on the device by the library's own offline prep, enough of them
     that their total exceeds 3x L2: rotating through them keeps every step's
     operands out of L2."""
     import svdquant_w4a4_gemm_b200 as sv
     from svdquant_w4a4_gemm_b200 import prep as dprep
-    d = workloads.draw_svdq(CASE)
+    case = CASE if case is None else case
+    d = workloads.draw_svdq(case)
     x0 = torch.from_numpy(d["x"]).to(dev).to(torch.bfloat16)
     W0 = torch.from_numpy(d["W"]).to(dev).to(torch.bfloat16)
     b0 = torch.from_numpy(d["bias"]).to(dev).to(torch.bfloat16)
     xc = torch.from_numpy(d["x_cal"]).to(dev).to(torch.bfloat16)
-    w0 = dprep.prepare_svdq(W0, b0, xc, CASE.r)
-    M, K, N, r = CASE.M, CASE.K, CASE.N, CASE.r
+    w0 = dprep.prepare_svdq(W0, b0, xc, case.r)
+    M, K, N, r = case.M, case.K, case.N, case.r
     gs = torch.empty(1, device=dev)
     sv.quantize_act(x0, w0.smooth, w0.L1t, None, out=(
         torch.empty(M, K // 2, dtype=torch.uint8, device=dev),
@@ -280,10 +281,47 @@ def bench_device(args, rank, world, dev):
     e2e_ms = a.elapsed_time(b) / e2e_steps
 
     del graph
-    legs = bench_awq_legs(sv, dev, l2) if args.legs and rank == 0 else None
+    legs = None
+    if args.legs and rank == 0:
+        legs = bench_awq_legs(sv, dev, l2)
+        legs.update(bench_gelu_leg(sv, dev, l2))
     return dict(steps=steps_done, total_ms=total_ms, k1_us=k1_us, k2_us=k2_us, clocks=clk.summary(), nsets=nsets,
                 set_mb=per / 2 ** 20, e2e_ms=e2e_ms, h2d=x_host.numel() * 2, d2h=y_host.numel() * 2,
                 legs=legs)
+
+
+def bench_gelu_leg(sv, dev, l2, steps=200, reps=5):
+    """The MLP up-projection GEMM (M4096 K3072 N12288 r32) with the plain
+    epilogue and with GELU(tanh) fused into it: device time per launch,
+    graphs over rotating sets > 3x L2."""
+    case = workloads.MLP_UP
+    sets, _ = make_sets(dev, l2, case)
+    for s in sets:
+        sv.quantize_act(s["x"], s["w"].smooth, s["w"].L1t, s["gs"], out=(s["q"], s["sf"], s["lora"], s["gso"]))
+    stream = torch.cuda.current_stream(dev)
+    cap = torch.cuda.Stream(dev)
+    out = {}
+    for act in (None, "gelu"):
+        g = torch.cuda.CUDAGraph()
+        cap.wait_stream(stream)
+        with torch.cuda.graph(g, stream=cap):
+            for i in range(steps):
+                s = sets[i % len(sets)]
+                sv.w4a4_linear(s["q"], s["sf"], s["gso"], s["lora"], s["w"], y=s["y"], act=act)
+        g.replay()
+        torch.cuda.synchronize(dev)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(reps):
+            g.replay()
+        b.record(stream)
+        torch.cuda.synchronize(dev)
+        us = a.elapsed_time(b) * 1e3 / (reps * steps)
+        fl = layer_flops(case.M, case.K, case.N, case.r)
+        out[f"mlp_up_gemm_{act or 'plain'}"] = {"us": round(us, 3), "TFLOP/s": round(fl / us / 1e6, 1)}
+        del g
+    sv.check_device_errors()
+    return out
 
 
 def bench_awq_legs(sv, dev, l2):

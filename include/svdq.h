@@ -142,6 +142,28 @@ svdq_status svdq_w4a4_linear(const uint8_t* q_act, const uint8_t* sf_act,
                              void* y_bf16, int64_t ldy, void* stream);
 
 /*
+ * svdq_w4a4_linear_act — svdq_w4a4_linear with an activation applied in
+ * the epilogue before the bf16 rounding (the fused GELU of the MLP
+ * up-projection; blog.margrop.com "技术细节 §2", GELU/MLP fusion):
+ *
+ *   y = bf16( act( dec(A)·dec(W)ᵀ + lora_act·L2 + bias ) )
+ *
+ *   activation  SVDQ_ACT_NONE (0): identity, the same as svdq_w4a4_linear;
+ *               SVDQ_ACT_GELU_TANH (1): 0.5·v·(1 + tanh(√(2/π)(v + 0.044715·v³)))
+ *               evaluated in fp32 with the hardware tanh approximation
+ *               (relative error about 2^-11, below the bf16 output rounding).
+ *   Other arguments and errors as svdq_w4a4_linear; an unknown activation
+ *   is INVALID_ARG.
+ */
+enum { SVDQ_ACT_NONE = 0, SVDQ_ACT_GELU_TANH = 1 };
+svdq_status svdq_w4a4_linear_act(const uint8_t* q_act, const uint8_t* sf_act,
+                                 const float* act_gscale, const float* lora_act,
+                                 const uint8_t* q_w, const uint8_t* sf_w, const float* w_gscale,
+                                 const void* L2t_bf16, int r, const void* bias_bf16,
+                                 int64_t M, int64_t N, int64_t K,
+                                 void* y_bf16, int64_t ldy, int activation, void* stream);
+
+/*
  * awq_w4a16_linear — int4-weight × bf16-activation linear for the
  * bandwidth-bound modulation layers (ainews.surl.tw paragraph 2;
  * app.hamidun.com "Что такое Nunchaku и SVDQuant"):

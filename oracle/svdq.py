@@ -124,8 +124,20 @@ def lora_down(x, s, L1t):
     return xh16 @ np.asarray(L1t, dtype=np.float64).T
 
 
-def svdq_linear(codes_a, sf_a, gs_a, xl, codes_w, sf_w, gs_w, L2t, bias):
-    """y = deq(A)·deq(W)ᵀ + xl·L2 + b, all in fp64.
+def gelu_tanh(v):
+    """GELU in its tanh form, 0.5·v·(1 + tanh(√(2/π)·(v + 0.044715·v³))), in fp64.
+
+    The MLP up-projection of a DiT block is followed by GELU(tanh); the
+    original engine fuses it into the GEMM (blog.margrop.com "技术细节 §2",
+    its per-architecture GELU/MLP fusion), which saves one round trip of
+    the layer's output through HBM.
+    """
+    v = np.asarray(v, dtype=np.float64)
+    return 0.5 * v * (1.0 + np.tanh(np.sqrt(2.0 / np.pi) * (v + 0.044715 * v * v * v)))
+
+
+def svdq_linear(codes_a, sf_a, gs_a, xl, codes_w, sf_w, gs_w, L2t, bias, act=None):
+    """y = act(deq(A)·deq(W)ᵀ + xl·L2 + b), all in fp64; act None or "gelu".
 
     codes_a [M, K], sf_a [M, K/16]; codes_w [N, K], sf_w [N, K/16];
     xl [M, r] (fp64 or fp32); L2t = L2ᵀ stored [N, r]; bias [N] or None.
@@ -137,11 +149,15 @@ def svdq_linear(codes_a, sf_a, gs_a, xl, codes_w, sf_w, gs_w, L2t, bias):
         y = y + np.asarray(xl, dtype=np.float64) @ np.asarray(L2t, dtype=np.float64).T
     if bias is not None:
         y = y + np.asarray(bias, dtype=np.float64)[None, :]
+    if act == "gelu":
+        y = gelu_tanh(y)
+    elif act is not None:
+        raise ValueError(f"unknown activation {act!r}")
     return y
 
 
-def svdq_forward(x, layer, gs_a=None):
-    """Whole layer from a bf16 activation: quantize, down-proj, GEMM.
+def svdq_forward(x, layer, gs_a=None, act=None):
+    """Whole layer from a bf16 activation: quantize, down-proj, GEMM (+ act).
 
     ``layer`` is the dict that ``oracle.prep.prepare_svdq_layer`` returns.
     """
@@ -149,5 +165,5 @@ def svdq_forward(x, layer, gs_a=None):
     r = layer["L1t"].shape[0]
     xl = lora_down(x, layer["s"], layer["L1t"]) if r else np.zeros((x.shape[0], 0))
     y = svdq_linear(q["codes"], q["sf"], q["gs"], xl, layer["codes_w"], layer["sf_w"],
-                    layer["gs_w"], layer["L2t"] if r else None, layer["bias"])
+                    layer["gs_w"], layer["L2t"] if r else None, layer["bias"], act=act)
     return dict(y=y, xl=xl, **q)

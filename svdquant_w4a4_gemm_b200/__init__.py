@@ -33,6 +33,8 @@ _SIGNATURES = {
     "svdq_quantize_act": (_int, [_vp, _i64, _i64, _i64, _vp, _vp, _int, _vp, _vp, _vp, _vp, _vp, _vp]),
     "svdq_w4a4_linear": (_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _int, _vp,
                                 _i64, _i64, _i64, _vp, _i64, _vp]),
+    "svdq_w4a4_linear_act": (_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _int, _vp,
+                                    _i64, _i64, _i64, _vp, _i64, _int, _vp]),
     "awq_w4a16_linear": (_int, [_vp, _i64, _i64, _vp, _vp, _vp, _vp, _int, _vp, _i64, _vp, _vp]),
     "svdq_check_device_errors": (_int, [_vp]),
     "svdq_set_wait_timeout_ns": (_u64, [_u64]),
@@ -136,22 +138,27 @@ class SvdqWeights:
         return self.q_w.shape[1] * 2
 
 
-def w4a4_linear(q, sf, gs_a, lora, w: SvdqWeights, *, y=None):
-    """y [M, N] bf16 = dec(q)·dec(W)ᵀ + lora·L2 + bias."""
+ACT_NONE, ACT_GELU_TANH = 0, 1
+_ACTS = {None: ACT_NONE, "gelu": ACT_GELU_TANH}
+
+
+def w4a4_linear(q, sf, gs_a, lora, w: SvdqWeights, *, y=None, act=None):
+    """y [M, N] bf16 = act(dec(q)·dec(W)ᵀ + lora·L2 + bias); act None or "gelu" (tanh form)."""
     M, K = q.shape[0], q.shape[1] * 2
     N, r = w.N, w.rank
     if y is None:
         y = torch.empty((M, N), dtype=torch.bfloat16, device=q.device)
-    _check(lib().svdq_w4a4_linear(_ptr(q), _ptr(sf), _ptr(gs_a), _ptr(lora) if r else None,
-                                  _ptr(w.q_w), _ptr(w.sf_w), _ptr(w.gs_w), _ptr(w.L2t) if r else None, r,
-                                  _ptr(w.bias), M, N, K, _ptr(y), y.stride(0), _stream(q.device)))
+    _check(lib().svdq_w4a4_linear_act(_ptr(q), _ptr(sf), _ptr(gs_a), _ptr(lora) if r else None,
+                                      _ptr(w.q_w), _ptr(w.sf_w), _ptr(w.gs_w),
+                                      _ptr(w.L2t) if r else None, r, _ptr(w.bias), M, N, K,
+                                      _ptr(y), y.stride(0), _ACTS[act], _stream(q.device)))
     return y
 
 
-def svdq_linear(x, w: SvdqWeights, gscale=None):
+def svdq_linear(x, w: SvdqWeights, gscale=None, act=None):
     """The whole layer: quantize_act then w4a4_linear (two kernels, same stream)."""
     q, sf, lora, gs = quantize_act(x, w.smooth, w.L1t if w.rank else None, gscale)
-    return w4a4_linear(q, sf, gs, lora, w)
+    return w4a4_linear(q, sf, gs, lora, w, act=act)
 
 
 def awq_w4a16_linear(x, act_scale_inv, qweight, scales, zeros, bias=None, *, y=None, group=64):

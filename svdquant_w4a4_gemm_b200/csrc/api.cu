@@ -225,6 +225,17 @@ svdq_status svdq_w4a4_linear(const uint8_t* q_act, const uint8_t* sf_act, const 
                              const float* w_gscale, const void* L2t_bf16, int r,
                              const void* bias_bf16, int64_t M, int64_t N, int64_t K, void* y_bf16,
                              int64_t ldy, void* stream) {
+  return svdq_w4a4_linear_act(q_act, sf_act, act_gscale, lora_act, q_w, sf_w, w_gscale, L2t_bf16, r,
+                              bias_bf16, M, N, K, y_bf16, ldy, SVDQ_ACT_NONE, stream);
+}
+
+svdq_status svdq_w4a4_linear_act(const uint8_t* q_act, const uint8_t* sf_act,
+                                 const float* act_gscale, const float* lora_act, const uint8_t* q_w,
+                                 const uint8_t* sf_w, const float* w_gscale, const void* L2t_bf16,
+                                 int r, const void* bias_bf16, int64_t M, int64_t N, int64_t K,
+                                 void* y_bf16, int64_t ldy, int activation, void* stream) {
+  if (activation != SVDQ_ACT_NONE && activation != SVDQ_ACT_GELU_TANH)
+    return fail(SVDQ_ERR_INVALID_ARG, "activation=%d must be 0 (none) or 1 (GELU tanh)", activation);
   if (!q_act || !sf_act || !act_gscale || !q_w || !sf_w || !w_gscale || !y_bf16)
     return fail(SVDQ_ERR_INVALID_ARG, "q_act, sf_act, act_gscale, q_w, sf_w, w_gscale and y must be non-null");
   if (M < 1 || M > (1ll << 30)) return fail(SVDQ_ERR_INVALID_ARG, "M=%lld out of range [1, 2^30]", (long long)M);
@@ -245,7 +256,7 @@ svdq_status svdq_w4a4_linear(const uint8_t* q_act, const uint8_t* sf_act, const 
   LaunchCtx ctx{};
   if (svdq_status e = device_ctx(stream, &ctx)) return e;
   if (svdq_status e = launch_w4a4_gemm(ctx, q_act, sf_act, act_gscale, lora_act, q_w, sf_w, w_gscale,
-                                       L2t_bf16, r, bias_bf16, M, N, K, y_bf16, ldy))
+                                       L2t_bf16, r, bias_bf16, M, N, K, y_bf16, ldy, activation))
     return e;
   return ok();
 }

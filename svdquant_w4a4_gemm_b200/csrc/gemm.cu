@@ -75,6 +75,16 @@ struct GemmParams {
   WaitCfg wait;
 };
 
+// GELU, tanh form, in fp32: 0.5·v·(1 + tanh(√(2/π)·(v + 0.044715·v³))).
+// The hardware tanh keeps the activation off the epilogue's critical path
+// (one MUFU op per element); its ~2^-11 relative error is below the bf16
+// rounding of the output that follows.
+__device__ __forceinline__ float gelu_tanh(float v) {
+  const float u = 0.7978845608028654f * fmaf(0.044715f * v, v * v, v);
+  const float h = 0.5f * v;
+  return fmaf(h, tanh_approx(u), h);
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&h);
@@ -110,7 +120,7 @@ __device__ __forceinline__ void tile_coords(int t, int tiles_n, int bn, int& m0,
   n0 = (t % tiles_n) * bn;
 }
 
-template <int BN>
+template <int BN, int ACT>
 __global__ void __launch_bounds__(kThreads, 1)
     w4a4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
                      const __grid_constant__ CUtensorMap tmap_b,
@@ -470,6 +480,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint16_t* bsl = bias_s + ew * BN;
     uint8_t* box = out_s + ew * L::kBoxBytes;
     uint8_t* brow = box + lane * 128;
+    constexpr bool gelu = ACT == SVDQ_ACT_GELU_TANH;
     int local = 0;                           // tiles drained
     for (int t = blockIdx.x; t < p.tiles; t += gridDim.x, ++local) {
       int m0, n0;
@@ -502,10 +513,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t bw[8] = {bb0.x, bb0.y, bb0.z, bb0.w, bb1.x, bb1.y, bb1.z, bb1.w};
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
-              const float lo = __fadd_rn(__fmul_rn(__uint_as_float(av[2 * e]), alpha),
-                                         __uint_as_float(bw[e] << 16));
-              const float hi = __fadd_rn(__fmul_rn(__uint_as_float(av[2 * e + 1]), alpha),
-                                         __uint_as_float(bw[e] & 0xFFFF0000u));
+              float lo = __fadd_rn(__fmul_rn(__uint_as_float(av[2 * e]), alpha),
+                                   __uint_as_float(bw[e] << 16));
+              float hi = __fadd_rn(__fmul_rn(__uint_as_float(av[2 * e + 1]), alpha),
+                                   __uint_as_float(bw[e] & 0xFFFF0000u));
+              if (gelu) {
+                lo = gelu_tanh(lo);
+                hi = gelu_tanh(hi);
+              }
               packed[(c + u) * 8 + e] = pack_bf16x2(lo, hi);
             }
           }
@@ -540,7 +555,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-template <int BN>
+template <int BN, int ACT>
 svdq_status launch_bn(const LaunchCtx& ctx, const CUtensorMap& ta, const CUtensorMap& tb,
                       const CUtensorMap& tl, const CUtensorMap& ty, const CUtensorMap& tr,
                       GemmParams p) {
@@ -549,14 +564,14 @@ svdq_status launch_bn(const LaunchCtx& ctx, const CUtensorMap& ta, const CUtenso
                       8 * (4 * kStages + 2 * kMaxRegions + 4) + 16;
   static bool attr_done[64] = {};
   if (!attr_done[ctx.device & 63]) {
-    cudaFuncSetAttribute(w4a4_gemm_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaFuncSetAttribute(w4a4_gemm_kernel<BN, ACT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          static_cast<int>(smem));
     attr_done[ctx.device & 63] = true;
   }
   p.tiles_n = (p.N + BN - 1) / BN;
   p.tiles = p.tiles_n * ((p.M + kBM - 1) / kBM);
   const int grid = std::min(p.tiles, ctx.num_sms);
-  w4a4_gemm_kernel<BN><<<grid, kThreads, smem, ctx.stream>>>(ta, tb, tl, ty, tr, p);
+  w4a4_gemm_kernel<BN, ACT><<<grid, kThreads, smem, ctx.stream>>>(ta, tb, tl, ty, tr, p);
   return check_launch("w4a4_gemm_kernel");
 }
 
@@ -566,7 +581,7 @@ svdq_status launch_w4a4_gemm(const LaunchCtx& ctx, const uint8_t* q_act, const u
                              const float* act_gscale, const float* lora_act, const uint8_t* q_w,
                              const uint8_t* sf_w, const float* w_gscale, const void* L2t, int r,
                              const void* bias, int64_t M, int64_t N, int64_t K, void* y,
-                             int64_t ldy) {
+                             int64_t ldy, int activation) {
   const int bn = (N % 192 == 0) ? 192 : 128;
   CUtensorMap ta{}, tb{}, tl{}, ty{}, tr{};
   if (!make_tmap_2d(&ta, q_act, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, M, K / 2, K / 2, kBM, kBKBytes,
@@ -604,8 +619,11 @@ svdq_status launch_w4a4_gemm(const LaunchCtx& ctx, const uint8_t* q_act, const u
   p.bias = static_cast<const uint16_t*>(bias);
   p.fault = ctx.fault_flags;
   p.wait = WaitCfg{ctx.timeout_ns, ctx.err_word};
-  return bn == 192 ? launch_bn<192>(ctx, ta, tb, tl, ty, tr, p)
-                   : launch_bn<128>(ctx, ta, tb, tl, ty, tr, p);
+  if (activation == SVDQ_ACT_GELU_TANH)
+    return bn == 192 ? launch_bn<192, SVDQ_ACT_GELU_TANH>(ctx, ta, tb, tl, ty, tr, p)
+                     : launch_bn<128, SVDQ_ACT_GELU_TANH>(ctx, ta, tb, tl, ty, tr, p);
+  return bn == 192 ? launch_bn<192, SVDQ_ACT_NONE>(ctx, ta, tb, tl, ty, tr, p)
+                   : launch_bn<128, SVDQ_ACT_NONE>(ctx, ta, tb, tl, ty, tr, p);
 }
 
 }  // namespace svdq

@@ -44,7 +44,7 @@ svdq_status launch_w4a4_gemm(const LaunchCtx& ctx, const uint8_t* q_act, const u
                              const float* act_gscale, const float* lora_act, const uint8_t* q_w,
                              const uint8_t* sf_w, const float* w_gscale, const void* L2t, int r,
                              const void* bias, int64_t M, int64_t N, int64_t K, void* y,
-                             int64_t ldy);
+                             int64_t ldy, int activation);
 
 svdq_status launch_awq_w4a16(const LaunchCtx& ctx, const void* x, int64_t M, int64_t K,
                              const float* act_scale_inv, const uint32_t* qweight,

@@ -13,7 +13,7 @@
 // work items and the load is balanced to one sub-tile.
 //   warp 0       TMA producer: x sub-tiles and the matching 64-column slices
 //                of L1ᵀ into a shared-memory ring as deep as shared memory
-//                allows (up to 12 sub-tiles: the loads come from HBM, and the
+//                allows, up to 8 sub-tiles (the loads come from HBM, and the
 //                ring must cover its latency).  The first loads of the ring
 //                are issued before the CTA-wide set-up, while
 //                the other warps compute RN(1/s) once for every column this
@@ -25,7 +25,13 @@
 //                sub-tiles in the same 128-row block ("segment").
 //   warps 2-9    quantizers, one sub-tile per warp (so up to 8 sub-tiles are
 //                worked on at once; with all warps on one sub-tile, each
-//                sub-tile costs a full dependent chain of latencies): lane l
+//                sub-tile costs a full dependent chain of latencies).  As many
+//                of them work as the ring has slots (at most 8), sub-tile i
+//                going to warp i mod slots: a warp then owns its ring slot,
+//                and the previous phase of every barrier it waits on is one
+//                it consumed itself (a parity wait cannot tell a phase from
+//                the one two before it, so a warp must never wait on a slot
+//                whose previous load may still be outstanding).  Lane l
 //                takes rows l, l+32, l+64, l+96 and each row's four 16-element
 //                groups: x̂ = x·inv_s, group max, E4M3 scale
 //                (cvt.rn.satfinite.e4m3x2; RN(gs / scale) from a per-CTA
@@ -49,8 +55,8 @@ namespace {
 
 constexpr int kBM = 128;
 constexpr int kSubK = 64;
-constexpr int kMaxStages = 12;
 constexpr int kQuantWarps = 8;   // one sub-tile each, so up to 8 in flight
+constexpr int kMaxStages = kQuantWarps;  // ring depth <= quantizer warps: one slot per warp
 constexpr int kEpiWarps = 4;
 constexpr int kThreads = 32 * (2 + kQuantWarps + kEpiWarps);
 constexpr uint32_t kXTileBytes = kBM * kSubK * 2;
@@ -58,7 +64,7 @@ constexpr uint32_t kXTileBytes = kBM * kSubK * 2;
 struct QuantParams {
   int M, K, r;
   int units;              // ceil(M/128) * (K/64) sub-tiles
-  int stages;             // ring depth, <= kMaxStages
+  int stages;             // ring depth, 2 .. kMaxStages; also the number of working quantizer warps
   const float* smooth_s;  // [K] or null
   const float* gs_in;     // static tensor scale, or null for dynamic
   const float* amax_src;  // dynamic: amax bits (written by the amax pass)
@@ -230,16 +236,16 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp < 2 + kQuantWarps) {
     // ------------------------------------------------------ quantizers ----
     const int qw = warp - 2;
-    // Each warp quantizes whole sub-tiles (units i = qw, qw + 8, ...), so up
-    // to 8 sub-tiles are in flight at once and each lane has 16 independent
-    // groups to interleave: lane l takes rows l, l + 32, l + 64, l + 96 of
-    // the tile, each row's four 16-element groups.
+    // Warp qw < ns quantizes whole sub-tiles (units i = qw, qw + ns, ...),
+    // all of them in ring slot qw, so up to ns sub-tiles are in flight at
+    // once and each lane has 16 independent groups to interleave: lane l
+    // takes rows l, l + 32, l + 64, l + 96 of the tile, each row's four
+    // 16-element groups.
     if (p.gs_copy && blockIdx.x == 0 && threadIdx.x == 64) *p.gs_copy = gs;
     const size_t kbytes = static_cast<size_t>(p.K) / 2;
-    for (int u = u0 + qw; u < u1; u += kQuantWarps) {
-      const int i = u - u0;
-      const int s = i % ns;
-      const uint32_t ph = (i / ns) & 1;
+    const int s = qw;
+    uint32_t ph = 0;
+    for (int u = u0 + qw; qw < ns && u < u1; u += ns, ph ^= 1u) {
       if (!mbar_wait(&full[s], ph, p.wait, kErrTimeoutFull)) break;
       const int rb = u / kblocks, kb = u % kblocks;
       const float* isk = inv_s + kb * kSubK;
@@ -401,7 +407,7 @@ constexpr size_t kSmemLimit = 227 * 1024;
 size_t quantize_fixed_bytes(int64_t K) {
   return 1024 + static_cast<size_t>(K) * 4 + 128 * 4 + 8 * (3 * kMaxStages + 4) + 16;
 }
-// Ring depth: as many sub-tiles as fit next to the RN(1/s) table, 2..12.
+// Ring depth: as many sub-tiles as fit next to the RN(1/s) table, 2..8.
 int quantize_stages(int64_t K, int r) {
   const size_t fixed = quantize_fixed_bytes(K);
   const size_t per = kXTileBytes + static_cast<size_t>(r) * 128;

@@ -62,6 +62,25 @@ def assert_gemm_close(y_gpu, y_ref, what=""):
     return mx, rel_f
 
 
+GELU_MAX_SLOPE = 1.129  # max |d/dv GELU_tanh(v)|, reached near v = 1.42
+
+
+def assert_gelu_close(y_gpu, y_ref, y_pre, what=""):
+    """The output bar through GELU: the epilogue's error before the activation
+    meets the plain bar, and GELU scales an error by at most its maximal slope,
+    so max|err| <= 1.129 · 2e-2 · rms(pre-activation); the Frobenius bar stays
+    relative to the GELU output itself, ||err||_F <= 5e-3·||ref||_F."""
+    y = y_gpu.float().cpu().numpy().astype(np.float64)
+    err = y - y_ref
+    rms_pre = np.sqrt(np.mean(np.asarray(y_pre, dtype=np.float64) ** 2))
+    rel_f = np.linalg.norm(err) / np.linalg.norm(y_ref)
+    mx = np.abs(err).max() / rms_pre
+    assert np.isfinite(y).all(), f"{what}: non-finite outputs"
+    assert mx <= GELU_MAX_SLOPE * 2e-2 and rel_f <= 5e-3, \
+        f"{what}: max|err|/rms(pre)={mx:.3e} relF={rel_f:.3e}"
+    return mx, rel_f
+
+
 def describe_byte_mismatch(got, ref):
     bad = np.nonzero(got != ref)[0]
     return f"{len(bad)} of {ref.size} bytes differ; first at {bad[:8].tolist()}: " \

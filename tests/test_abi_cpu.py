@@ -23,7 +23,8 @@ def _declared_functions():
 def test_library_exports_every_declared_function():
     L = sv.lib()
     names = _declared_functions()
-    assert {"svdq_quantize_act", "svdq_w4a4_linear", "awq_w4a16_linear"} <= set(names)
+    assert {"svdq_quantize_act", "svdq_w4a4_linear", "svdq_w4a4_linear_act",
+            "awq_w4a16_linear"} <= set(names)
     for n in names:
         assert hasattr(L, n), n
 
@@ -70,6 +71,10 @@ def test_linear_and_awq_validation_is_host_side():
     st = L.svdq_w4a4_linear(v(16), v(16), v(16), None, v(16), v(16), v(16), None, 0, None,
                             4, 32, 64, v(16), 30, None)
     assert st == sv.INVALID_ARG  # ldy % 8
+    st = L.svdq_w4a4_linear_act(v(16), v(16), v(16), None, v(16), v(16), v(16), None, 0, None,
+                                4, 32, 64, v(16), 32, 2, None)
+    assert st == sv.INVALID_ARG  # unknown activation
+    assert b"activation=2" in L.svdq_last_error_detail()
     st = L.awq_w4a16_linear(v(16), 9, 64, None, v(16), v(16), v(16), 64, None, 32, v(16), None)
     assert st == sv.INVALID_ARG  # M > 8
     st = L.awq_w4a16_linear(v(16), 1, 64, None, v(16), v(16), v(16), 128, None, 32, v(16), None)

@@ -21,7 +21,7 @@ import torch
 
 import workloads
 from oracle import prep, svdq as osv
-from tests._gpu import (assert_gemm_close, bf16, f32, needs_gpu, prepared, u8,
+from tests._gpu import (assert_gelu_close, assert_gemm_close, bf16, f32, needs_gpu, prepared, u8,
                         weights_from_layer)
 
 import svdquant_w4a4_gemm_b200 as sv
@@ -29,14 +29,18 @@ import svdquant_w4a4_gemm_b200 as sv
 pytestmark = [pytest.mark.gpu, needs_gpu]
 
 
-def _gemm_on_oracle_inputs(case, smooth=True, with_bias=True):
+def _gemm_on_oracle_inputs(case, smooth=True, with_bias=True, act=None, bias=None):
     d, L = prepared(case, smooth=smooth, with_bias=with_bias)
-    out = osv.svdq_forward(d["x"], L)
+    if bias is not None:
+        L = dict(L, bias=bias)
+    out = osv.svdq_forward(d["x"], L, act=act)
     w = weights_from_layer(L)
     r = case.r
     lora = f32(out["xl"]) if r else None
-    y = sv.w4a4_linear(u8(out["packed"]), u8(out["sf_swizzled"]), f32([out["gs"]]), lora, w)
+    y = sv.w4a4_linear(u8(out["packed"]), u8(out["sf_swizzled"]), f32([out["gs"]]), lora, w, act=act)
     torch.cuda.synchronize()
+    if act is not None:
+        return y, out["y"], osv.svdq_forward(d["x"], L)["y"]
     return y, out["y"]
 
 
@@ -85,6 +89,26 @@ def test_zero_residual_gives_low_rank_branch_only():
     assert_gemm_close(y, ref, "R = 0")
 
 
+# GELU(tanh) in the epilogue: both tile widths, a ragged M and N tail
+@pytest.mark.parametrize("M,K,N,r", [(256, 512, 512, 32), (200, 512, 384, 16), (77, 320, 400, 64)])
+def test_gemm_gelu_small(M, K, N, r):
+    case = workloads.small_case(M, K, N, r, seed=M * 5 + N + r)
+    y, ref, pre = _gemm_on_oracle_inputs(case, act="gelu")
+    assert_gelu_close(y, ref, pre, f"GELU M{M} K{K} N{N} r{r}")
+
+
+def test_gemm_gelu_saturating_range():
+    # a bias ramp over [-12, 12] pushes the pre-activations through the
+    # negative tail (GELU -> 0), the bend near 0 and the linear regime
+    M, K, N, r = 256, 512, 384, 32
+    case = workloads.small_case(M, K, N, r, seed=41)
+    ramp = workloads.to_bf16(np.linspace(-12.0, 12.0, N).astype(np.float32))
+    y, ref, pre = _gemm_on_oracle_inputs(case, act="gelu", bias=ramp)
+    assert_gelu_close(y, ref, pre, "GELU over [-12, 12]")
+    yn = y.float().cpu().numpy()
+    assert (yn[:, :N // 8] <= 0).all() and (yn[:, :N // 8] > -0.2).all()  # far negative: tiny, non-positive
+
+
 def test_whole_layer_tiny_workload():
     case = workloads.TINY
     d, L = prepared(case)
@@ -119,13 +143,15 @@ def _full(case_name, r):
     return d, L
 
 
-def _whole_layer_sampled(d, L, x=None, step=16):
+def _whole_layer_sampled(d, L, x=None, step=16, act=None):
     x = d["x"] if x is None else x
     gs = osv.act_tensor_scale(x, L["s"])
-    y = sv.svdq_linear(bf16(x), weights_from_layer(L), f32([gs]))
+    y = sv.svdq_linear(bf16(x), weights_from_layer(L), f32([gs]), act=act)
     torch.cuda.synchronize()
     rows = np.arange(0, x.shape[0], step)
-    ref = osv.svdq_forward(x[rows], L, gs)["y"]
+    ref = osv.svdq_forward(x[rows], L, gs, act=act)["y"]
+    if act is not None:
+        return y[torch.from_numpy(rows).cuda()], ref, osv.svdq_forward(x[rows], L, gs)["y"]
     return y[torch.from_numpy(rows).cuda()], ref
 
 
@@ -139,6 +165,13 @@ def test_mlp_up_full_size():
     d, L = _full(workloads.MLP_UP.name, 32)
     y, ref = _whole_layer_sampled(d, L, step=32)
     assert_gemm_close(y, ref, "mlp up full")
+
+
+def test_mlp_up_gelu_full_size():
+    # the MLP up-projection as a DiT block runs it: GELU(tanh) fused into the epilogue
+    d, L = _full(workloads.MLP_UP.name, 32)
+    y, ref, pre = _whole_layer_sampled(d, L, step=32, act="gelu")
+    assert_gelu_close(y, ref, pre, "mlp up + GELU full")
 
 
 def test_mlp_down_full_size():

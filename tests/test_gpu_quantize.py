@@ -96,6 +96,37 @@ def test_quantize_mlp_down_full_size_sampled():
     assert np.linalg.norm(lora[rows] - xl_ref) <= 1e-4 * np.linalg.norm(xl_ref)
 
 
+# the ring depth follows K and r (as many 16 KB sub-tiles as shared memory
+# holds, at most 8): 8 at K=3072 for r <= 64, 6 at r=128; 7 and 5 at
+# K=12288 for r = 64 and 128.  Repeated runs must give the same bytes every
+# time: a sub-tile quantized from a slot that does not yet hold it changes
+# the codes of that run only.
+@pytest.mark.parametrize("M,K,r", [(4608, 3072, 128), (4608, 3072, 32), (4096, 12288, 64),
+                                   (4096, 12288, 128), (1000, 3072, 0)])
+def test_quantize_repeatable_at_every_ring_depth(M, K, r):
+    rng = np.random.default_rng(M + K + r)
+    x = workloads.to_bf16(rng.standard_normal((M, K)).astype(np.float32))
+    s = rng.uniform(0.5, 4.0, K).astype(np.float32)
+    L1t = workloads.to_bf16(rng.standard_normal((max(r, 16), K)).astype(np.float32) * 0.05)
+    L = dict(s=s, L1t=L1t)
+    gs_ref = osv.act_tensor_scale(x, s)
+    q0, sf0, lora0, _ = _run(x, L, r, False, gs_ref)
+    for _ in range(8):
+        q, sf, lora, _ = _run(x, L, r, False, gs_ref)
+        assert np.array_equal(q, q0), "codes: " + describe_byte_mismatch(q.ravel(), q0.ravel())
+        assert np.array_equal(sf, sf0), "scales: " + describe_byte_mismatch(sf, sf0)
+        if r:
+            assert np.abs(lora - lora0).max() <= 1e-4 * np.sqrt(np.mean(lora0.astype(np.float64) ** 2))
+    rows = np.arange(0, M, 7)
+    ref = osv.quantize_act(x[rows], s, gs_ref)
+    assert np.array_equal(q0[rows], ref["packed"])
+    from oracle import codecs
+    assert np.array_equal(codecs.unswizzle_scales(sf0, M, K // 16)[rows], ref["sf"])
+    if r:
+        xl_ref = osv.lora_down(x[rows], s, L1t[:r])
+        assert np.linalg.norm(lora0[rows] - xl_ref) <= 1e-4 * np.linalg.norm(xl_ref)
+
+
 def test_quantize_strided_rows_and_gs_copy():
     case = workloads.small_case(160, 256, 64, 32, seed=5)
     d, L = prepared(case)

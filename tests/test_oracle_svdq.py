@@ -108,6 +108,48 @@ def test_svdq_linear_equals_triple_loop_on_tiny_shapes():
     np.testing.assert_allclose(got, ref, rtol=1e-12, atol=1e-12)
 
 
+def test_gelu_tanh_special_values_and_identities():
+    g = svdq.gelu_tanh
+    assert g(0.0) == 0.0
+    # tanh is odd, so g(v) - g(-v) = v exactly in real arithmetic
+    v = np.linspace(-9, 9, 361)
+    np.testing.assert_allclose(g(v) - g(-v), v, rtol=0, atol=1e-13)
+    # saturated tails: the identity above and the zero tail
+    assert abs(g(30.0) - 30.0) < 1e-12 and abs(g(-30.0)) < 1e-12
+    # slope 1/2 at the origin, from the series g(v) = v/2 + c·v²/2 + O(v⁴), c = √(2/π)
+    h = 1e-6
+    assert abs((g(h) - g(-h)) / (2 * h) - 0.5) < 1e-9
+    assert abs((g(h) + g(-h)) / (h * h) - np.sqrt(2 / np.pi)) < 1e-5
+
+
+def test_gelu_tanh_is_the_tanh_form_and_close_to_exact_gelu():
+    import math
+    import torch
+    v = np.linspace(-8, 8, 2001)
+    lib = torch.nn.functional.gelu(torch.from_numpy(v), approximate="tanh").numpy()
+    np.testing.assert_allclose(svdq.gelu_tanh(v), lib, rtol=1e-14, atol=1e-15)
+    exact = np.array([0.5 * t * (1 + math.erf(t / math.sqrt(2))) for t in v])
+    err = np.abs(svdq.gelu_tanh(v) - exact)
+    assert err.max() < 1e-3 and err.max() > 1e-5  # an approximation of Φ, not Φ itself
+
+
+def test_gelu_is_applied_after_the_bias():
+    rng = _rng(9)
+    M, K, N, r = 2, 32, 3, 1
+    ca = rng.integers(0, 16, (M, K)).astype(np.uint8)
+    cw = rng.integers(0, 16, (N, K)).astype(np.uint8)
+    sfa = rng.integers(0, 0x7F, (M, K // 16)).astype(np.uint8)
+    sfw = rng.integers(0, 0x7F, (N, K // 16)).astype(np.uint8)
+    xl, L2t, bias = rng.standard_normal((M, r)), rng.standard_normal((N, r)), rng.standard_normal(N) * 5
+    pre = _brute_y(ca, sfa, 3.0, xl, cw, sfw, 5.0, L2t, bias)
+    got = svdq.svdq_linear(ca, sfa, np.float32(3), xl, cw, sfw, np.float32(5), L2t, bias, act="gelu")
+    import math
+    want = np.vectorize(lambda t: 0.5 * t * (1 + math.tanh(math.sqrt(2 / math.pi) * (t + 0.044715 * t ** 3))))(pre)
+    np.testing.assert_allclose(got, want, rtol=1e-12, atol=1e-12)
+    with pytest.raises(ValueError):
+        svdq.svdq_linear(ca, sfa, np.float32(3), xl, cw, sfw, np.float32(5), L2t, bias, act="relu")
+
+
 def test_lora_down_equals_loop_over_k():
     rng = _rng(7)
     x = workloads.to_bf16(rng.standard_normal((3, 48)).astype(np.float32))
