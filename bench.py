@@ -285,9 +285,57 @@ def bench_device(args, rank, world, dev):
     if args.legs and rank == 0:
         legs = bench_awq_legs(sv, dev, l2)
         legs.update(bench_gelu_leg(sv, dev, l2))
+        try:
+            legs.update(bench_dynamic_scale_leg(sv, dev, sets, gsteps, capture))
+        except Exception as e:  # noqa: BLE001 - report it on the line, keep the line
+            legs["quantize_dynamic_error"] = str(e)[:200]
     return dict(steps=steps_done, total_ms=total_ms, k1_us=k1_us, k2_us=k2_us, clocks=clk.summary(), nsets=nsets,
                 set_mb=per / 2 ** 20, e2e_ms=e2e_ms, h2d=x_host.numel() * 2, d2h=y_host.numel() * 2,
                 legs=legs)
+
+
+def bench_dynamic_scale_leg(sv, dev, sets, gsteps, capture, reps=5):
+    """The headline activation quantized three ways: static gs_a (the
+    step's K1), dynamic gs_a by a max pass + K1 + finalize, and dynamic gs_a
+    in one cooperative launch.  Device time per call over rotating sets."""
+    stream = torch.cuda.current_stream(dev)
+    ws = [torch.zeros(sv.QUANTIZE_WORKSPACE_BYTES, dtype=torch.uint8, device=dev) for _ in sets]
+    for s_ in sets:
+        s_["gdyn"] = torch.empty(1, device=dev)
+    bodies = {
+        "static": lambda s_: sv.quantize_act(s_["x"], s_["w"].smooth, s_["w"].L1t, s_["gs"],
+                                             out=(s_["q"], s_["sf"], s_["lora"], s_["gso"])),
+        "dynamic_max_pass": lambda s_: sv.quantize_act(s_["x"], s_["w"].smooth, s_["w"].L1t, None,
+                                                       out=(s_["q"], s_["sf"], s_["lora"], s_["gdyn"])),
+    }
+    idx = {id(s_): i for i, s_ in enumerate(sets)}
+    bodies["dynamic_single_pass"] = lambda s_: sv.quantize_act_dynamic(
+        s_["x"], s_["w"].smooth, s_["w"].L1t, out=(s_["q"], s_["sf"], s_["lora"], s_["gdyn"]),
+        workspace=ws[idx[id(s_)]])
+    out = {}
+    for name, body in bodies.items():
+        for i in range(3):
+            body(sets[i % len(sets)])
+        try:
+            g = capture(body)
+            how = "graph"
+        except Exception:            # a launch kind the stream capture refuses: time it eagerly
+            torch.cuda.synchronize(dev)
+            g, how = None, "eager"
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(reps):
+            if g is not None:
+                g.replay()
+            else:
+                for i in range(gsteps):
+                    body(sets[i % len(sets)])
+        b.record(stream)
+        torch.cuda.synchronize(dev)
+        out[f"quantize_{name}"] = {"us": round(a.elapsed_time(b) * 1e3 / (reps * gsteps), 3), "timed": how}
+        del g
+    sv.check_device_errors()
+    return out
 
 
 def bench_gelu_leg(sv, dev, l2, steps=200, reps=5):

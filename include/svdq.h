@@ -109,6 +109,33 @@ svdq_status svdq_quantize_act(const void* x_bf16, int64_t M, int64_t K, int64_t 
                               void* stream);
 
 /*
+ * svdq_quantize_act_dynamic — svdq_quantize_act with the dynamic tensor scale
+ * gs_a = 2688 / max|x̂| (1 if that max is 0) computed inside the same kernel
+ * (one launch instead of a max pass, the quantize kernel and a finalize
+ * step).  Every CTA first reads its share of x for the max, the CTAs then
+ * meet at a grid-wide barrier, and the quantization reads x again (from L2
+ * at these sizes).  Outputs are bit-identical to svdq_quantize_act with
+ * act_gscale = NULL.
+ *
+ *   act_gscale_out  fp32 device scalar, receives gs_a.  Required.
+ *   workspace   SVDQ_QUANTIZE_WORKSPACE_BYTES of device memory, 16-byte
+ *               aligned, owned by the caller; the call clears it before its
+ *               kernel runs and leaves unspecified contents.  Calls that may
+ *               overlap on the GPU must use distinct workspaces.
+ *   Other arguments as svdq_quantize_act.
+ *   The kernel is a cooperative launch (all CTAs resident at once: at most
+ *   one per SM); its grid barrier waits at most the library's wait bound
+ *   (svdq_set_wait_timeout_ns), after which svdq_check_device_errors
+ *   reports SVDQ_ERR_DEVICE_TIMEOUT (bit 16) and the outputs are undefined.
+ *   Errors: INVALID_ARG, MISALIGNED, UNSUPPORTED_DEVICE, CUDA.
+ */
+#define SVDQ_QUANTIZE_WORKSPACE_BYTES 16
+svdq_status svdq_quantize_act_dynamic(const void* x_bf16, int64_t M, int64_t K, int64_t ldx,
+                                      const float* smooth_s, const void* L1t_bf16, int r,
+                                      float* act_gscale_out, void* workspace, uint8_t* q_out,
+                                      uint8_t* sf_out, float* lora_out, void* stream);
+
+/*
  * svdq_w4a4_linear — the 4-bit GEMM with the low-rank up-projection fused
  * ("the low-rank up-projection is fused with the 4-bit compute kernel",
  * blog.margrop.com "技术细节 §1" step 4):
@@ -164,6 +191,33 @@ svdq_status svdq_w4a4_linear_act(const uint8_t* q_act, const uint8_t* sf_act,
                                  void* y_bf16, int64_t ldy, int activation, void* stream);
 
 /*
+ * svdq_w4a4_linear_split — the fused projection with its output stored in
+ * `parts` separate buffers: the fused QKV projection (blog.margrop.com
+ * "技术细节 §2": the original engine fuses the Q, K and V projections),
+ * one quantized activation, one GEMM over the concatenated weight
+ * [W_q; W_k; W_v], and Q, K and V written straight to their own tensors.
+ *
+ *   y = bf16( act( dec(A)·dec(W)ᵀ + lora_act·L2 + bias ) )        [M, N]
+ *   columns [i·N/parts, (i+1)·N/parts) of y  ->  y_parts[i], [M, N/parts]
+ *
+ *   parts     1, 2 or 3.  N/parts must be a multiple of 128 when parts > 1
+ *             (an output tile never straddles two parts).
+ *   y_parts   HOST array of `parts` device pointers, each 16-byte aligned
+ *             and row-major with leading dimension ldy; the array is read
+ *             during the call only.
+ *   ldy       >= N/parts, a multiple of 8.
+ *   Other arguments and errors as svdq_w4a4_linear_act; parts == 1 is that
+ *   call.
+ */
+svdq_status svdq_w4a4_linear_split(const uint8_t* q_act, const uint8_t* sf_act,
+                                   const float* act_gscale, const float* lora_act,
+                                   const uint8_t* q_w, const uint8_t* sf_w, const float* w_gscale,
+                                   const void* L2t_bf16, int r, const void* bias_bf16,
+                                   int64_t M, int64_t N, int64_t K, int parts,
+                                   void* const* y_parts, int64_t ldy, int activation,
+                                   void* stream);
+
+/*
  * awq_w4a16_linear — int4-weight × bf16-activation linear for the
  * bandwidth-bound modulation layers (ainews.surl.tw paragraph 2;
  * app.hamidun.com "Что такое Nunchaku и SVDQuant"):
@@ -211,8 +265,10 @@ uint64_t svdq_set_wait_timeout_ns(uint64_t ns);
 /*
  * svdq_debug_set_fault — TEST HOOK.  flags = 1 makes the next launches of
  * svdq_w4a4_linear skip one producer arrive so that the consumer's bounded
- * wait runs out (host-side fault injection; nothing traps or faults).
- * 0 clears it.  Returns the previous flags.
+ * wait runs out; flags = 2 makes the first CTA of the next
+ * svdq_quantize_act_dynamic launches skip its arrival at the grid barrier so
+ * that the other CTAs' bounded waits run out (host-side fault injection;
+ * nothing traps or faults).  0 clears it.  Returns the previous flags.
  */
 int svdq_debug_set_fault(int flags);
 

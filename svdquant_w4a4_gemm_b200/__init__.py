@@ -31,10 +31,14 @@ _SIGNATURES = {
     "svdq_last_error_detail": (ctypes.c_char_p, []),
     "svdq_nvfp4_scale_bytes": (_sz, [_i64, _i64]),
     "svdq_quantize_act": (_int, [_vp, _i64, _i64, _i64, _vp, _vp, _int, _vp, _vp, _vp, _vp, _vp, _vp]),
+    "svdq_quantize_act_dynamic": (_int, [_vp, _i64, _i64, _i64, _vp, _vp, _int, _vp, _vp, _vp, _vp,
+                                         _vp, _vp]),
     "svdq_w4a4_linear": (_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _int, _vp,
                                 _i64, _i64, _i64, _vp, _i64, _vp]),
     "svdq_w4a4_linear_act": (_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _int, _vp,
                                     _i64, _i64, _i64, _vp, _i64, _int, _vp]),
+    "svdq_w4a4_linear_split": (_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _int, _vp,
+                                      _i64, _i64, _i64, _int, _vp, _i64, _int, _vp]),
     "awq_w4a16_linear": (_int, [_vp, _i64, _i64, _vp, _vp, _vp, _vp, _int, _vp, _i64, _vp, _vp]),
     "svdq_check_device_errors": (_int, [_vp]),
     "svdq_set_wait_timeout_ns": (_u64, [_u64]),
@@ -114,6 +118,34 @@ def quantize_act(x, smooth=None, L1t=None, gscale=None, *, out=None):
     return q, sf, lora, gs
 
 
+QUANTIZE_WORKSPACE_BYTES = 16
+
+
+def quantize_act_dynamic(x, smooth=None, L1t=None, *, out=None, workspace=None):
+    """quantize_act with the dynamic tensor scale computed in the same kernel
+    (one cooperative launch with a grid barrier).  ``workspace``: a device
+    buffer of at least QUANTIZE_WORKSPACE_BYTES bytes, 16-byte aligned (one is
+    allocated if None); calls that may overlap on the GPU need their own."""
+    assert x.dtype == torch.bfloat16 and x.dim() == 2 and x.stride(1) == 1
+    M, K = x.shape
+    r = 0 if L1t is None else L1t.shape[0]
+    dev = x.device
+    if out is None:
+        q = torch.empty((M, K // 2), dtype=torch.uint8, device=dev)
+        sf = torch.empty((scale_bytes(M, K),), dtype=torch.uint8, device=dev)
+        lora = torch.empty((M, r), dtype=torch.float32, device=dev) if r else None
+        gs = torch.empty((1,), dtype=torch.float32, device=dev)
+    else:
+        q, sf, lora, gs = out
+    if workspace is None:
+        workspace = torch.empty((QUANTIZE_WORKSPACE_BYTES,), dtype=torch.uint8, device=dev)
+    assert workspace.numel() * workspace.element_size() >= QUANTIZE_WORKSPACE_BYTES
+    _check(lib().svdq_quantize_act_dynamic(_ptr(x), M, K, x.stride(0), _ptr(smooth), _ptr(L1t), r,
+                                           _ptr(gs), _ptr(workspace), _ptr(q), _ptr(sf), _ptr(lora),
+                                           _stream(dev)))
+    return q, sf, lora, gs
+
+
 @dataclass
 class SvdqWeights:
     """Prepared weights of one W4A4 layer (all on the device)."""
@@ -153,6 +185,25 @@ def w4a4_linear(q, sf, gs_a, lora, w: SvdqWeights, *, y=None, act=None):
                                       _ptr(w.L2t) if r else None, r, _ptr(w.bias), M, N, K,
                                       _ptr(y), y.stride(0), _ACTS[act], _stream(q.device)))
     return y
+
+
+def w4a4_linear_split(q, sf, gs_a, lora, w: SvdqWeights, parts=3, *, ys=None, act=None):
+    """The fused projection stored as ``parts`` outputs [M, N/parts] bf16 (Q, K, V of a
+    fused QKV projection): columns [i·N/parts, (i+1)·N/parts) of y go to ys[i]."""
+    M, K = q.shape[0], q.shape[1] * 2
+    N, r = w.N, w.rank
+    n_part = N // parts
+    if ys is None:
+        ys = [torch.empty((M, n_part), dtype=torch.bfloat16, device=q.device) for _ in range(parts)]
+    ys = list(ys)
+    ldy = ys[0].stride(0)
+    assert len(ys) == parts and all(t.stride(0) == ldy and t.stride(1) == 1 for t in ys)
+    arr = (_vp * parts)(*[_ptr(t) for t in ys])
+    _check(lib().svdq_w4a4_linear_split(_ptr(q), _ptr(sf), _ptr(gs_a), _ptr(lora) if r else None,
+                                        _ptr(w.q_w), _ptr(w.sf_w), _ptr(w.gs_w),
+                                        _ptr(w.L2t) if r else None, r, _ptr(w.bias), M, N, K, parts,
+                                        ctypes.cast(arr, _vp), ldy, _ACTS[act], _stream(q.device)))
+    return tuple(ys)
 
 
 def svdq_linear(x, w: SvdqWeights, gscale=None, act=None):

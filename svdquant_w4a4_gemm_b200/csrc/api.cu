@@ -187,10 +187,11 @@ size_t svdq_nvfp4_scale_bytes(int64_t rows, int64_t K) {
   return static_cast<size_t>(rp * cp);
 }
 
-svdq_status svdq_quantize_act(const void* x_bf16, int64_t M, int64_t K, int64_t ldx,
+namespace {
+svdq_status quantize_entry(const void* x_bf16, int64_t M, int64_t K, int64_t ldx,
                               const float* smooth_s, const void* L1t_bf16, int r,
                               const float* act_gscale, float* act_gscale_out, uint8_t* q_out,
-                              uint8_t* sf_out, float* lora_out, void* stream) {
+                              uint8_t* sf_out, float* lora_out, uint32_t* grid_sync, void* stream) {
   if (!x_bf16 || !q_out || !sf_out) return fail(SVDQ_ERR_INVALID_ARG, "x, q_out and sf_out must be non-null");
   if (M < 1 || M > (1ll << 30)) return fail(SVDQ_ERR_INVALID_ARG, "M=%lld out of range [1, 2^30]", (long long)M);
   if (K < 64 || K % 64 != 0 || K > (1ll << 20))
@@ -202,7 +203,7 @@ svdq_status svdq_quantize_act(const void* x_bf16, int64_t M, int64_t K, int64_t 
     return fail(SVDQ_ERR_INVALID_ARG, "r > 0 needs L1t_bf16 and lora_out");
   if (!act_gscale && !act_gscale_out)
     return fail(SVDQ_ERR_INVALID_ARG, "dynamic scale (act_gscale == NULL) needs act_gscale_out");
-  if (quantize_smem_bytes(K, r) > 227 * 1024)
+  if (quantize_smem_bytes(K, r) > 227 * 1024 - 64)  // the opt-in limit less the static words
     return fail(SVDQ_ERR_INVALID_ARG, "K=%lld with r=%d needs more than 227 KB of shared memory "
                 "(about K <= 24800 at r = 128, 37100 at r = 32)", (long long)K, r);
   if (!aligned16(x_bf16) || !aligned16(q_out) || !aligned16(sf_out) ||
@@ -215,9 +216,29 @@ svdq_status svdq_quantize_act(const void* x_bf16, int64_t M, int64_t K, int64_t 
   LaunchCtx ctx{};
   if (svdq_status e = device_ctx(stream, &ctx)) return e;
   if (svdq_status e = launch_quantize_act(ctx, x_bf16, M, K, ldx, smooth_s, L1t_bf16, r, act_gscale,
-                                          act_gscale_out, q_out, sf_out, lora_out))
+                                          act_gscale_out, q_out, sf_out, lora_out, grid_sync))
     return e;
   return ok();
+}
+}  // namespace
+
+svdq_status svdq_quantize_act(const void* x_bf16, int64_t M, int64_t K, int64_t ldx,
+                              const float* smooth_s, const void* L1t_bf16, int r,
+                              const float* act_gscale, float* act_gscale_out, uint8_t* q_out,
+                              uint8_t* sf_out, float* lora_out, void* stream) {
+  return quantize_entry(x_bf16, M, K, ldx, smooth_s, L1t_bf16, r, act_gscale, act_gscale_out, q_out,
+                        sf_out, lora_out, nullptr, stream);
+}
+
+svdq_status svdq_quantize_act_dynamic(const void* x_bf16, int64_t M, int64_t K, int64_t ldx,
+                                      const float* smooth_s, const void* L1t_bf16, int r,
+                                      float* act_gscale_out, void* workspace, uint8_t* q_out,
+                                      uint8_t* sf_out, float* lora_out, void* stream) {
+  if (!act_gscale_out || !workspace)
+    return fail(SVDQ_ERR_INVALID_ARG, "act_gscale_out and workspace must be non-null");
+  if (!aligned16(workspace)) return fail(SVDQ_ERR_MISALIGNED, "workspace must be 16-byte aligned");
+  return quantize_entry(x_bf16, M, K, ldx, smooth_s, L1t_bf16, r, nullptr, act_gscale_out, q_out,
+                        sf_out, lora_out, static_cast<uint32_t*>(workspace), stream);
 }
 
 svdq_status svdq_w4a4_linear(const uint8_t* q_act, const uint8_t* sf_act, const float* act_gscale,
@@ -234,21 +255,41 @@ svdq_status svdq_w4a4_linear_act(const uint8_t* q_act, const uint8_t* sf_act,
                                  const uint8_t* sf_w, const float* w_gscale, const void* L2t_bf16,
                                  int r, const void* bias_bf16, int64_t M, int64_t N, int64_t K,
                                  void* y_bf16, int64_t ldy, int activation, void* stream) {
+  void* const parts[1] = {y_bf16};
+  return svdq_w4a4_linear_split(q_act, sf_act, act_gscale, lora_act, q_w, sf_w, w_gscale, L2t_bf16,
+                                r, bias_bf16, M, N, K, 1, parts, ldy, activation, stream);
+}
+
+svdq_status svdq_w4a4_linear_split(const uint8_t* q_act, const uint8_t* sf_act,
+                                   const float* act_gscale, const float* lora_act,
+                                   const uint8_t* q_w, const uint8_t* sf_w, const float* w_gscale,
+                                   const void* L2t_bf16, int r, const void* bias_bf16, int64_t M,
+                                   int64_t N, int64_t K, int parts, void* const* y_parts,
+                                   int64_t ldy, int activation, void* stream) {
   if (activation != SVDQ_ACT_NONE && activation != SVDQ_ACT_GELU_TANH)
     return fail(SVDQ_ERR_INVALID_ARG, "activation=%d must be 0 (none) or 1 (GELU tanh)", activation);
-  if (!q_act || !sf_act || !act_gscale || !q_w || !sf_w || !w_gscale || !y_bf16)
+  if (parts < 1 || parts > 3) return fail(SVDQ_ERR_INVALID_ARG, "parts=%d must be 1, 2 or 3", parts);
+  if (!y_parts) return fail(SVDQ_ERR_INVALID_ARG, "y_parts must be non-null");
+  for (int i = 0; i < parts; ++i)
+    if (!y_parts[i]) return fail(SVDQ_ERR_INVALID_ARG, "y_parts[%d] must be non-null", i);
+  if (!q_act || !sf_act || !act_gscale || !q_w || !sf_w || !w_gscale)
     return fail(SVDQ_ERR_INVALID_ARG, "q_act, sf_act, act_gscale, q_w, sf_w, w_gscale and y must be non-null");
   if (M < 1 || M > (1ll << 30)) return fail(SVDQ_ERR_INVALID_ARG, "M=%lld out of range [1, 2^30]", (long long)M);
   if (N < 16 || N % 16 != 0 || N > (1ll << 30))
     return fail(SVDQ_ERR_INVALID_ARG, "N=%lld must be a positive multiple of 16", (long long)N);
+  if (parts > 1 && N % (128ll * parts) != 0)
+    return fail(SVDQ_ERR_INVALID_ARG, "N=%lld: N/parts must be a multiple of 128 for parts=%d",
+                (long long)N, parts);
   if (K < 64 || K % 64 != 0 || K > (1ll << 20))
     return fail(SVDQ_ERR_INVALID_ARG, "K=%lld must be a positive multiple of 64 (<= 2^20)", (long long)K);
-  if (ldy < N || ldy % 8 != 0)
-    return fail(SVDQ_ERR_INVALID_ARG, "ldy=%lld must be >= N and a multiple of 8", (long long)ldy);
+  if (ldy < N / parts || ldy % 8 != 0)
+    return fail(SVDQ_ERR_INVALID_ARG, "ldy=%lld must be >= N/parts and a multiple of 8", (long long)ldy);
   if (!valid_rank(r)) return fail(SVDQ_ERR_INVALID_ARG, "rank r=%d must be 0, 16, 32, 64 or 128", r);
   if (r > 0 && (!lora_act || !L2t_bf16)) return fail(SVDQ_ERR_INVALID_ARG, "r > 0 needs lora_act and L2t_bf16");
+  bool ys_aligned = true;
+  for (int i = 0; i < parts; ++i) ys_aligned = ys_aligned && aligned16(y_parts[i]);
   if (!aligned16(q_act) || !aligned16(sf_act) || !aligned16(q_w) || !aligned16(sf_w) ||
-      !aligned16(y_bf16) || (r > 0 && (!aligned16(L2t_bf16) || !aligned16(lora_act))))
+      !ys_aligned || (r > 0 && (!aligned16(L2t_bf16) || !aligned16(lora_act))))
     return fail(SVDQ_ERR_MISALIGNED, "codes, scales, lora_act, L2t and y must be 16-byte aligned");
   if ((reinterpret_cast<uintptr_t>(act_gscale) & 3) || (reinterpret_cast<uintptr_t>(w_gscale) & 3) ||
       (bias_bf16 && (reinterpret_cast<uintptr_t>(bias_bf16) & 1)))
@@ -256,7 +297,8 @@ svdq_status svdq_w4a4_linear_act(const uint8_t* q_act, const uint8_t* sf_act,
   LaunchCtx ctx{};
   if (svdq_status e = device_ctx(stream, &ctx)) return e;
   if (svdq_status e = launch_w4a4_gemm(ctx, q_act, sf_act, act_gscale, lora_act, q_w, sf_w, w_gscale,
-                                       L2t_bf16, r, bias_bf16, M, N, K, y_bf16, ldy, activation))
+                                       L2t_bf16, r, bias_bf16, M, N, K, parts, y_parts, ldy,
+                                       activation))
     return e;
   return ok();
 }
@@ -300,7 +342,7 @@ svdq_status svdq_check_device_errors(void* stream) {
   if (word) {
     cudaMemset(ctx.err_word, 0, sizeof(uint32_t));
     return fail(SVDQ_ERR_DEVICE_TIMEOUT, "device error word 0x%x (1 data wait, 2 slot wait, 4 "
-                "accumulator wait, 8 drain)", word);
+                "accumulator wait, 8 drain, 16 grid barrier)", word);
   }
   return ok();
 }

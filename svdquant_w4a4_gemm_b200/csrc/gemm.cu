@@ -42,9 +42,11 @@
 //               columns of hi and 32 of lo (bf16 of xl·gs_a·gs_w and of its
 //               remainder), swizzled by hand.
 //   warps 7-10  epilogue, one per quadrant: per 64-column box, TMEM ->
-//               registers (α·acc + bias -> bf16) -> a 32 x 64 staging box in
-//               shared memory -> TMA store (full-line writes, clipped at the
-//               M and N edges); then release the accumulator.
+//               registers (α·acc + bias [-> GELU] -> bf16) -> a 32 x 64
+//               staging box in shared memory -> TMA store (full-line writes,
+//               clipped at the M and N edges) into the tile's output (one,
+//               or one of up to three parts: Q, K, V of a fused
+//               projection); then release the accumulator.
 #include "internal.h"
 #include "ptx.cuh"
 
@@ -71,6 +73,7 @@ struct GemmParams {
   const float* gs_a;
   const float* gs_w;
   const uint16_t* bias;   // [N] or null
+  int n_part;             // split output: columns per part (tmap_y, tmap_y1, tmap_y2); 0 = one output
   int fault;              // test hook: 1 = the first ring slot never fills
   WaitCfg wait;
 };
@@ -126,7 +129,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                      const __grid_constant__ CUtensorMap tmap_b,
                      const __grid_constant__ CUtensorMap tmap_l2,
                      const __grid_constant__ CUtensorMap tmap_y,
-                     const __grid_constant__ CUtensorMap tmap_lr, const GemmParams p) {
+                     const __grid_constant__ CUtensorMap tmap_lr,
+                     const __grid_constant__ CUtensorMap tmap_y1,
+                     const __grid_constant__ CUtensorMap tmap_y2, const GemmParams p) {
   using L = Layout<BN>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -486,6 +491,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       int m0, n0;
       tile_coords(t, p.tiles_n, BN, m0, n0);
       const int a = local & 1;
+      // the output this tile goes to (a tile never straddles two parts)
+      const CUtensorMap* ymap = &tmap_y;
+      int ycol = n0;
+      if (p.n_part) {
+        const int part = n0 / p.n_part;
+        ycol = n0 - part * p.n_part;
+        ymap = part == 0 ? &tmap_y : (part == 1 ? &tmap_y1 : &tmap_y2);
+      }
       // the tile's bias columns into this warp's shared-memory copy
       for (int c = lane; c < BN; c += 32) {
         const int col = n0 + c;
@@ -540,7 +553,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) {
-          tma_store_2d(&tmap_y, box, n0 + 64 * j, m0 + 32 * quad);
+          tma_store_2d(ymap, box, ycol + 64 * j, m0 + 32 * quad);
           bulk_commit_group();
         }
       }
@@ -558,7 +571,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 template <int BN, int ACT>
 svdq_status launch_bn(const LaunchCtx& ctx, const CUtensorMap& ta, const CUtensorMap& tb,
                       const CUtensorMap& tl, const CUtensorMap& ty, const CUtensorMap& tr,
-                      GemmParams p) {
+                      const CUtensorMap& ty1, const CUtensorMap& ty2, GemmParams p) {
   using L = Layout<BN>;
   const size_t smem = 1024 + static_cast<size_t>(L::kRing) + kEpiWarps * L::kBoxBytes + L::kBias +
                       8 * (4 * kStages + 2 * kMaxRegions + 4) + 16;
@@ -571,7 +584,7 @@ svdq_status launch_bn(const LaunchCtx& ctx, const CUtensorMap& ta, const CUtenso
   p.tiles_n = (p.N + BN - 1) / BN;
   p.tiles = p.tiles_n * ((p.M + kBM - 1) / kBM);
   const int grid = std::min(p.tiles, ctx.num_sms);
-  w4a4_gemm_kernel<BN, ACT><<<grid, kThreads, smem, ctx.stream>>>(ta, tb, tl, ty, tr, p);
+  w4a4_gemm_kernel<BN, ACT><<<grid, kThreads, smem, ctx.stream>>>(ta, tb, tl, ty, tr, ty1, ty2, p);
   return check_launch("w4a4_gemm_kernel");
 }
 
@@ -580,10 +593,12 @@ svdq_status launch_bn(const LaunchCtx& ctx, const CUtensorMap& ta, const CUtenso
 svdq_status launch_w4a4_gemm(const LaunchCtx& ctx, const uint8_t* q_act, const uint8_t* sf_act,
                              const float* act_gscale, const float* lora_act, const uint8_t* q_w,
                              const uint8_t* sf_w, const float* w_gscale, const void* L2t, int r,
-                             const void* bias, int64_t M, int64_t N, int64_t K, void* y,
-                             int64_t ldy, int activation) {
-  const int bn = (N % 192 == 0) ? 192 : 128;
-  CUtensorMap ta{}, tb{}, tl{}, ty{}, tr{};
+                             const void* bias, int64_t M, int64_t N, int64_t K, int parts,
+                             void* const* y_parts, int64_t ldy, int activation) {
+  // the tile width must divide every part (parts > 1: N/parts is a multiple of 128)
+  const int64_t n_part = N / parts;
+  const int bn = (n_part % 192 == 0) ? 192 : 128;
+  CUtensorMap ta{}, tb{}, tl{}, ty{}, tr{}, ty1{}, ty2{};
   if (!make_tmap_2d(&ta, q_act, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, M, K / 2, K / 2, kBM, kBKBytes,
                     128))
     return SVDQ_ERR_CUDA;
@@ -604,9 +619,12 @@ svdq_status launch_w4a4_gemm(const LaunchCtx& ctx, const uint8_t* q_act, const u
   } else {
     tr = ta;
   }
-  if (!make_tmap_2d(&ty, y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, M, N, static_cast<uint64_t>(ldy) * 2,
-                    32, 64, 128))
-    return SVDQ_ERR_CUDA;
+  CUtensorMap* ymaps[3] = {&ty, &ty1, &ty2};
+  for (int i = 0; i < parts; ++i)
+    if (!make_tmap_2d(ymaps[i], y_parts[i], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, M, n_part,
+                      static_cast<uint64_t>(ldy) * 2, 32, 64, 128))
+      return SVDQ_ERR_CUDA;
+  for (int i = parts; i < 3; ++i) *ymaps[i] = ty;
   GemmParams p{};
   p.M = static_cast<int>(M);
   p.N = static_cast<int>(N);
@@ -617,13 +635,14 @@ svdq_status launch_w4a4_gemm(const LaunchCtx& ctx, const uint8_t* q_act, const u
   p.gs_a = act_gscale;
   p.gs_w = w_gscale;
   p.bias = static_cast<const uint16_t*>(bias);
+  p.n_part = parts > 1 ? static_cast<int>(n_part) : 0;
   p.fault = ctx.fault_flags;
   p.wait = WaitCfg{ctx.timeout_ns, ctx.err_word};
   if (activation == SVDQ_ACT_GELU_TANH)
-    return bn == 192 ? launch_bn<192, SVDQ_ACT_GELU_TANH>(ctx, ta, tb, tl, ty, tr, p)
-                     : launch_bn<128, SVDQ_ACT_GELU_TANH>(ctx, ta, tb, tl, ty, tr, p);
-  return bn == 192 ? launch_bn<192, SVDQ_ACT_NONE>(ctx, ta, tb, tl, ty, tr, p)
-                   : launch_bn<128, SVDQ_ACT_NONE>(ctx, ta, tb, tl, ty, tr, p);
+    return bn == 192 ? launch_bn<192, SVDQ_ACT_GELU_TANH>(ctx, ta, tb, tl, ty, tr, ty1, ty2, p)
+                     : launch_bn<128, SVDQ_ACT_GELU_TANH>(ctx, ta, tb, tl, ty, tr, ty1, ty2, p);
+  return bn == 192 ? launch_bn<192, SVDQ_ACT_NONE>(ctx, ta, tb, tl, ty, tr, ty1, ty2, p)
+                   : launch_bn<128, SVDQ_ACT_NONE>(ctx, ta, tb, tl, ty, tr, ty1, ty2, p);
 }
 
 }  // namespace svdq

@@ -38,13 +38,13 @@ size_t quantize_smem_bytes(int64_t K, int r);
 svdq_status launch_quantize_act(const LaunchCtx& ctx, const void* x, int64_t M, int64_t K,
                                 int64_t ldx, const float* smooth_s, const void* L1t, int r,
                                 const float* act_gscale, float* act_gscale_out, uint8_t* q_out,
-                                uint8_t* sf_out, float* lora_out);
+                                uint8_t* sf_out, float* lora_out, uint32_t* grid_sync = nullptr);
 
 svdq_status launch_w4a4_gemm(const LaunchCtx& ctx, const uint8_t* q_act, const uint8_t* sf_act,
                              const float* act_gscale, const float* lora_act, const uint8_t* q_w,
                              const uint8_t* sf_w, const float* w_gscale, const void* L2t, int r,
-                             const void* bias, int64_t M, int64_t N, int64_t K, void* y,
-                             int64_t ldy, int activation);
+                             const void* bias, int64_t M, int64_t N, int64_t K, int parts,
+                             void* const* y_parts, int64_t ldy, int activation);
 
 svdq_status launch_awq_w4a16(const LaunchCtx& ctx, const void* x, int64_t M, int64_t K,
                              const float* act_scale_inv, const uint32_t* qweight,

@@ -16,6 +16,7 @@ enum : uint32_t {
   kErrTimeoutEmpty = 1u << 1,  // a producer gave up waiting for a free slot
   kErrTimeoutAcc = 1u << 2,    // the epilogue gave up waiting for the MMA
   kErrTimeoutDrain = 1u << 3,  // draining in-flight copies gave up
+  kErrTimeoutGrid = 1u << 4,   // a CTA gave up waiting for the others at a grid barrier
 };
 
 struct WaitCfg {
@@ -96,6 +97,35 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const 
 // Bring the 128-byte line holding `p` into L1 (no register result).
 __device__ __forceinline__ void prefetch_l1(const void* p) {
   asm volatile("prefetch.global.L1 [%0];" ::"l"(reinterpret_cast<uint64_t>(p)));
+}
+
+__device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t* p) {
+  uint32_t v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+// Named barrier over `threads` threads (a multiple of 32) of the CTA.
+__device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t threads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
+
+// One thread per CTA: arrive at a grid-wide barrier (a counter that is zero
+// at launch) and wait, bounded, until `expected` CTAs have arrived.  Only for
+// kernels whose CTAs are all resident at once (cooperative launch).
+__device__ __forceinline__ bool grid_arrive_wait(uint32_t* ctr, uint32_t expected, const WaitCfg& w) {
+  __threadfence();  // this CTA's writes before its arrival
+  atomicAdd(ctr, 1u);
+  if (ld_acquire_gpu(ctr) >= expected) return true;
+  const uint64_t t0 = globaltimer();
+  while (ld_acquire_gpu(ctr) < expected) {
+    if (globaltimer() - t0 > w.timeout_ns) {
+      atomicOr(w.err, kErrTimeoutGrid);
+      return false;
+    }
+    __nanosleep(64);
+  }
+  return true;
 }
 
 // hardware tanh (one MUFU op), relative error about 2^-11

@@ -45,6 +45,16 @@
 //                the accumulator.
 // HBM traffic is the algorithmic minimum: x once, codes + scales + xl once;
 // L1ᵀ slices come from L2.
+//
+// Single-pass dynamic scale (gs_a = 2688 / max|x̂| computed in the same
+// launch): every CTA first streams its sub-tiles once for the max (phase A;
+// the quantizer warps take the sub-tiles as in phase B and release each
+// slot straight away), folds its max into a global word, and meets the
+// other CTAs at a grid barrier (cooperative launch, bounded wait); then
+// phase B quantizes as above with the tensor-wide gs_a, reading x again,
+// now from L2 (the CTA's phase-B loads go out while it waits at the
+// barrier).  The ring runs through both phases as one sequence of 2n
+// items, item i in slot i mod ns, owned by quantizer warp i mod ns.
 #include <cstdio>
 
 #include "internal.h"
@@ -72,6 +82,8 @@ struct QuantParams {
   uint8_t* q_out;
   uint8_t* sf_out;
   float* lora_out;
+  uint32_t* sync;         // single-pass dynamic scale: [0] CTAs arrived, [1] max|x̂| bits, zero at launch
+  int fault;              // test hook: bit 2 = CTA 0 never arrives at the grid barrier
   WaitCfg wait;
 };
 
@@ -93,7 +105,9 @@ __device__ __forceinline__ void unit_range(int units, int& u0, int& u1) {
   u1 = static_cast<int>((static_cast<int64_t>(blockIdx.x + 1) * units) / gridDim.x);
 }
 
-__global__ void __launch_bounds__(kThreads, 1)
+// 14 warps: four of them share some SM sub-partition, whose 16 K registers
+// then allow at most 128 a thread
+__global__ void __maxnreg__(128)
     quantize_act_kernel(const __grid_constant__ CUtensorMap tmap_x,
                         const __grid_constant__ CUtensorMap tmap_l1, const QuantParams p) {
   extern __shared__ uint8_t smem_raw[];
@@ -118,6 +132,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem_cols = p.r <= 16 ? 32u : static_cast<uint32_t>(2 * p.r);
   int u0, u1;
   unit_range(p.units, u0, u1);
+  // ring items: phase A (single-pass dynamic scale only), then phase B
+  const int n_units = u1 - u0;
+  const int phase_b0 = p.sync ? n_units : 0;   // first phase-B item
+  const int n_items = phase_b0 + n_units;
 
   // Warp 0 sets up the barriers and issues the first ns loads right
   // away; the rest of the CTA fills the RN(1/s) and RN(gs/scale) tables in
@@ -135,12 +153,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     fence_mbar_init();
     tma_prefetch_desc(&tmap_x);
     if (has_lr) tma_prefetch_desc(&tmap_l1);
-    for (int u = u0; u < min(u1, u0 + ns); ++u) {
-      const int s = u - u0;
+    for (int i = 0; i < min(n_items, ns); ++i) {
+      const int u = u0 + (i < n_units ? i : i - n_units);
+      const bool l1 = has_lr && i >= phase_b0;
       const int rb = u / kblocks, kb = u % kblocks;
-      mbar_arrive_expect_tx(&full[s], kXTileBytes + (has_lr ? l1_bytes : 0u));
-      tma_load_2d(xs + s * kXTileBytes, &tmap_x, &full[s], kb * kSubK, rb * kBM);
-      if (has_lr) tma_load_2d(ls + s * l1_bytes, &tmap_l1, &full[s], kb * kSubK, 0);
+      mbar_arrive_expect_tx(&full[i], kXTileBytes + (l1 ? l1_bytes : 0u));
+      tma_load_2d(xs + i * kXTileBytes, &tmap_x, &full[i], kb * kSubK, rb * kBM);
+      if (l1) tma_load_2d(ls + i * l1_bytes, &tmap_l1, &full[i], kb * kSubK, 0);
     }
   }
   if (warp != 0) {
@@ -161,9 +180,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_relinquish();
   }
   // RN(gs / dec(sf)) for every finite E4M3 scale code (0 for the zero
-  // scale): one IEEE division per code per CTA instead of one per group
-  const float gs = p.gs_in ? *p.gs_in : tensor_scale_from_amax(*p.amax_src);
-  if (threadIdx.x < 128) {
+  // scale): one IEEE division per code per CTA instead of one per group.
+  // Single-pass dynamic scale: gs is known only after phase A.
+  __shared__ uint32_t cta_amax_bits;
+  __shared__ float gs_shared;
+  __shared__ int grid_ok;
+  if (threadIdx.x == 0) {
+    cta_amax_bits = 0u;
+    grid_ok = 1;
+  }
+  const float gs = p.sync ? 1.0f : (p.gs_in ? *p.gs_in : tensor_scale_from_amax(*p.amax_src));
+  if (threadIdx.x < 128 && !p.sync) {
     const float d = e4m3_to_f32(threadIdx.x);
     gs_over_d[threadIdx.x] = (d == 0.0f || threadIdx.x == 127) ? 0.0f : __fdiv_rn(gs, d);
   }
@@ -175,16 +202,17 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0) {
     // ------------------------------------------------------- producer ----
     if (lane == 0) {
-      int issued = min(u1 - u0, ns);  // issued before the set-up sync
-      for (int u = u0 + ns; u < u1; ++u) {
-        const int i = u - u0;
+      int issued = min(n_items, ns);  // issued before the set-up sync
+      for (int i = ns; i < n_items; ++i) {
         const int s = i % ns;
         const uint32_t ph = (i / ns) & 1;
         if (!mbar_wait(&empty[s], ph ^ 1, p.wait, kErrTimeoutEmpty)) break;
+        const int u = u0 + (i < n_units ? i : i - n_units);
+        const bool l1 = has_lr && i >= phase_b0;
         const int rb = u / kblocks, kb = u % kblocks;
-        mbar_arrive_expect_tx(&full[s], kXTileBytes + (has_lr ? l1_bytes : 0u));
+        mbar_arrive_expect_tx(&full[s], kXTileBytes + (l1 ? l1_bytes : 0u));
         tma_load_2d(xs + s * kXTileBytes, &tmap_x, &full[s], kb * kSubK, rb * kBM);
-        if (has_lr) tma_load_2d(ls + s * l1_bytes, &tmap_l1, &full[s], kb * kSubK, 0);
+        if (l1) tma_load_2d(ls + s * l1_bytes, &tmap_l1, &full[s], kb * kSubK, 0);
         issued = i + 1;
       }
       // never leave the CTA with a copy still landing in its shared memory
@@ -202,15 +230,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint64_t db0 = make_sdesc(smem_u32(ls), 16, 1024, kSwz128);
       int seg = 0;             // segments started by this CTA
       bool first = true;       // first sub-tile of the current segment
-      int s = 0;               // ring slot of unit u
-      uint32_t ph = 0;         // its phase parity
+      int s = phase_b0 % ns;   // ring slot of unit u's phase-B item
+      uint32_t qd_par = 0;     // per slot: parity of its next qdone phase
       int kb = u0 % kblocks;   // 64-column block of unit u
       for (int u = u0; u < u1; ++u) {
         const int buf = seg & 1;
         if (first && seg >= 2 &&
             !mbar_wait(&acc_empty[buf], ((seg >> 1) - 1) & 1, p.wait, kErrTimeoutAcc))
           break;
-        if (!mbar_wait(&qdone[s], ph, p.wait, kErrTimeoutFull)) break;
+        if (!mbar_wait(&qdone[s], (qd_par >> s) & 1u, p.wait, kErrTimeoutFull)) break;
+        qd_par ^= 1u << s;
         tc_fence_after();
         const uint64_t da = da0 + ((static_cast<uint32_t>(s) * kXTileBytes) >> 4);
         const uint64_t db = db0 + ((static_cast<uint32_t>(s) * l1_bytes) >> 4);
@@ -220,10 +249,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int kk = 1; kk < kSubK / 16; ++kk) umma_f16(d, da + 2 * kk, db + 2 * kk, idesc, 1u);
         umma_commit(&empty[s]);
         first = false;
-        if (++s == ns) {
-          s = 0;
-          ph ^= 1u;
-        }
+        if (++s == ns) s = 0;
         const bool seg_end = (u + 1 == u1) || (kb + 1 == kblocks);  // the row block ends
         kb = kb + 1 == kblocks ? 0 : kb + 1;
         if (seg_end) {
@@ -241,12 +267,81 @@ __global__ void __launch_bounds__(kThreads, 1)
     // once and each lane has 16 independent groups to interleave: lane l
     // takes rows l, l + 32, l + 64, l + 96 of the tile, each row's four
     // 16-element groups.
-    if (p.gs_copy && blockIdx.x == 0 && threadIdx.x == 64) *p.gs_copy = gs;
     const size_t kbytes = static_cast<size_t>(p.K) / 2;
     const int s = qw;
     uint32_t ph = 0;
-    for (int u = u0 + qw; qw < ns && u < u1; u += ns, ph ^= 1u) {
-      if (!mbar_wait(&full[s], ph, p.wait, kErrTimeoutFull)) break;
+    int i = qw;              // ring item
+    float gsq = gs;
+    if (p.sync) {
+      // phase A: max|x·inv_s| over this warp's sub-tiles; each slot is
+      // released as soon as it is read
+      bool ok = true;
+      float m8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      for (; qw < ns && i < phase_b0; i += ns, ph ^= 1u) {
+        // one verdict per warp: lanes that disagree at the time limit must not split up
+        if (!__all_sync(0xffffffffu, mbar_wait(&full[s], ph, p.wait, kErrTimeoutFull))) {
+          ok = false;
+          break;
+        }
+        const float* isk = inv_s + ((u0 + i) % kblocks) * kSubK;
+#pragma unroll 2
+        for (int j = 0; j < 4; ++j) {
+          const int row = lane + 32 * j;
+          const uint8_t* trow = xs + s * kXTileBytes + row * 128;
+#pragma unroll
+          for (int g = 0; g < 4; ++g) {
+            const uint4 v0 = *reinterpret_cast<const uint4*>(trow + (((2 * g) ^ (row & 7)) << 4));
+            const uint4 v1 = *reinterpret_cast<const uint4*>(trow + (((2 * g + 1) ^ (row & 7)) << 4));
+            const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+            const float4* is4 = reinterpret_cast<const float4*>(isk + 16 * g);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              const float4 iv = is4[q];
+              m8[2 * q] = fmaxf(m8[2 * q], fabsf(__fmul_rn(bf16lo(w[2 * q]), iv.x)));
+              m8[2 * q] = fmaxf(m8[2 * q], fabsf(__fmul_rn(bf16hi(w[2 * q]), iv.y)));
+              m8[2 * q + 1] = fmaxf(m8[2 * q + 1], fabsf(__fmul_rn(bf16lo(w[2 * q + 1]), iv.z)));
+              m8[2 * q + 1] = fmaxf(m8[2 * q + 1], fabsf(__fmul_rn(bf16hi(w[2 * q + 1]), iv.w)));
+            }
+          }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[s]);
+      }
+      float am = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
+                       fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, o));
+      if (lane == 0) {
+        atomicMax(&cta_amax_bits, __float_as_uint(am));  // non-negative floats order like their bits
+        if (!ok) grid_ok = 0;
+      }
+      named_bar_sync(1, 32 * kQuantWarps);
+      if (qw == 0 && lane == 0) {
+        // one thread per CTA: fold the CTA's max in, then wait for every CTA
+        atomicMax(&p.sync[1], cta_amax_bits);
+        const bool skip = (p.fault & 2) && blockIdx.x == 0;  // test hook: this CTA never arrives
+        const bool arrived = !skip && grid_arrive_wait(&p.sync[0], gridDim.x, p.wait);
+        const float g = tensor_scale_from_amax(__uint_as_float(ld_acquire_gpu(&p.sync[1])));
+        gs_shared = g;
+        if (!arrived) grid_ok = 0;
+        if (arrived && blockIdx.x == 0 && p.gs_copy) *p.gs_copy = g;
+      }
+      named_bar_sync(1, 32 * kQuantWarps);
+      gsq = gs_shared;
+      if (threadIdx.x - 64 < 128) {  // the RN(gs / dec(sf)) table, now that gs is known
+        const uint32_t c = threadIdx.x - 64;
+        const float d = e4m3_to_f32(c);
+        gs_over_d[c] = (d == 0.0f || c == 127) ? 0.0f : __fdiv_rn(gsq, d);
+      }
+      const bool cta_ok = grid_ok != 0;
+      named_bar_sync(1, 32 * kQuantWarps);
+      if (!cta_ok) i = n_items;  // the barrier or a wait failed: quantize nothing
+    } else if (p.gs_copy && blockIdx.x == 0 && threadIdx.x == 64) {
+      *p.gs_copy = gs;
+    }
+    for (; qw < ns && i < n_items; i += ns, ph ^= 1u) {
+      const int u = u0 + i - phase_b0;
+      if (!__all_sync(0xffffffffu, mbar_wait(&full[s], ph, p.wait, kErrTimeoutFull))) break;
       const int rb = u / kblocks, kb = u % kblocks;
       const float* isk = inv_s + kb * kSubK;
       uint8_t* sfb = p.sf_out + (static_cast<size_t>(rb) * kblocks + kb) * 512 + lane * 16;
@@ -281,7 +376,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int e = 0; e < 4; ++e) m8[e] = fmaxf(m8[e], m8[e + 4]);
           const float amax = fmaxf(fmaxf(m8[0], m8[2]), fmaxf(m8[1], m8[3]));
-          const float t = __fmul_rn(__fdiv_rn(amax, 6.0f), gs);
+          const float t = __fmul_rn(__fdiv_rn(amax, 6.0f), gsq);
           const uint32_t sf = cvt_e4m3(t);
           const float inv = gs_over_d[sf & 127u];  // RN(gs / dec(sf)); 0 for a zero scale
           sfw |= sf << (8 * g);
@@ -403,7 +498,7 @@ __global__ void act_scale_finalize_kernel(float* gs) {
 }  // namespace
 
 namespace {
-constexpr size_t kSmemLimit = 227 * 1024;
+constexpr size_t kSmemLimit = 227 * 1024 - 64;  // less the kernel's static shared words
 size_t quantize_fixed_bytes(int64_t K) {
   return 1024 + static_cast<size_t>(K) * 4 + 128 * 4 + 8 * (3 * kMaxStages + 4) + 16;
 }
@@ -424,7 +519,7 @@ size_t quantize_smem_bytes(int64_t K, int r) {
 svdq_status launch_quantize_act(const LaunchCtx& ctx, const void* x, int64_t M, int64_t K,
                                 int64_t ldx, const float* smooth_s, const void* L1t, int r,
                                 const float* act_gscale, float* act_gscale_out, uint8_t* q_out,
-                                uint8_t* sf_out, float* lora_out) {
+                                uint8_t* sf_out, float* lora_out, uint32_t* grid_sync) {
   CUtensorMap tx{}, tl{};
   if (!make_tmap_2d(&tx, x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, M, K, ldx * 2, kBM, kSubK, 128))
     return SVDQ_ERR_CUDA;
@@ -441,9 +536,14 @@ svdq_status launch_quantize_act(const LaunchCtx& ctx, const void* x, int64_t M, 
   p.stages = quantize_stages(K, r);
   p.smooth_s = smooth_s;
   p.gs_in = act_gscale;
-  p.amax_src = act_gscale ? nullptr : act_gscale_out;
-  p.gs_copy = (act_gscale && act_gscale_out && act_gscale_out != act_gscale) ? act_gscale_out
-                                                                              : nullptr;
+  const bool single_pass = !act_gscale && grid_sync;
+  p.amax_src = (act_gscale || single_pass) ? nullptr : act_gscale_out;
+  p.gs_copy = single_pass ? act_gscale_out
+                          : ((act_gscale && act_gscale_out && act_gscale_out != act_gscale)
+                                 ? act_gscale_out
+                                 : nullptr);
+  p.sync = single_pass ? grid_sync : nullptr;
+  p.fault = ctx.fault_flags;
   p.q_out = q_out;
   p.sf_out = sf_out;
   p.lora_out = lora_out;
@@ -452,7 +552,10 @@ svdq_status launch_quantize_act(const LaunchCtx& ctx, const void* x, int64_t M, 
   cudaStream_t st = ctx.stream;
   if (r > 0 && cudaMemsetAsync(lora_out, 0, static_cast<size_t>(M) * r * 4, st) != cudaSuccess)
     return check_launch("memset lora_out");
-  if (!act_gscale) {
+  if (single_pass) {
+    if (cudaMemsetAsync(grid_sync, 0, 2 * sizeof(uint32_t), st) != cudaSuccess)
+      return check_launch("memset workspace");
+  } else if (!act_gscale) {
     if (cudaMemsetAsync(act_gscale_out, 0, 4, st) != cudaSuccess) return check_launch("memset gs");
     const int bx = static_cast<int>((K / 8 + 255) / 256);
     const int by = static_cast<int>(std::min<int64_t>(M, std::max(1, 4 * ctx.num_sms / bx)));
@@ -464,10 +567,29 @@ svdq_status launch_quantize_act(const LaunchCtx& ctx, const void* x, int64_t M, 
   static bool attr_done[64] = {};
   if (!attr_done[ctx.device & 63]) {
     cudaFuncSetAttribute(quantize_act_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         227 * 1024);
+                         static_cast<int>(kSmemLimit));
     attr_done[ctx.device & 63] = true;
   }
   const int grid = std::min(p.units, ctx.num_sms);
+  if (single_pass) {
+    // the CTAs meet at a grid barrier: all of them must be resident at once
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, quantize_act_kernel, tx, tl, p);
+    if (e != cudaSuccess) {
+      cudaGetLastError();
+      return fail(SVDQ_ERR_CUDA, "quantize_act_kernel (cooperative): %s", cudaGetErrorString(e));
+    }
+    return SVDQ_OK;
+  }
   quantize_act_kernel<<<grid, kThreads, smem, st>>>(tx, tl, p);
   if (svdq_status e = check_launch("quantize_act_kernel")) return e;
   if (!act_gscale) {

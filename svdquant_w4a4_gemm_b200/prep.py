@@ -45,6 +45,20 @@ def prepare_svdq(W, bias, x_cal, r, smooth=True):
                        bias=None if bias is None else bias.contiguous())
 
 
+def prepare_svdq_fused(Ws, biases, x_cal, r, smooth=True):
+    """One prepared layer for projections that read the same input (Q, K and V
+    of an attention block): their weights stacked along N, [W_0; W_1; ...],
+    smoothed, decomposed and quantized together, so one activation
+    quantization serves all of them.  The output columns of part i are
+    [Σ_{j<i} N_j, Σ_{j<=i} N_j); ``w4a4_linear_split`` stores them apart."""
+    W = torch.cat(list(Ws), dim=0)
+    bias = None
+    if any(b is not None for b in biases):
+        bias = torch.cat([b if b is not None else torch.zeros(Wi.shape[0], dtype=W.dtype, device=W.device)
+                          for Wi, b in zip(Ws, biases)])
+    return prepare_svdq(W, bias, x_cal, r, smooth=smooth)
+
+
 def prepare_awq(W, x_cal, group=64):
     """W [N, K] bf16, x_cal [*, K] -> (act_scale_inv [K] fp32, qweight [N, K/8] int32,
     scales [N, K/64] fp16, zeros [N, K/64] fp16)."""

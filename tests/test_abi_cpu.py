@@ -62,6 +62,19 @@ def test_quantize_validation_is_host_side():
     assert b"K=96" in sv.lib().svdq_last_error_detail() or True
 
 
+def test_single_pass_dynamic_quantize_validation_is_host_side():
+    L = sv.lib()
+    v = ctypes.c_void_p
+    st = L.svdq_quantize_act_dynamic(v(16), 4, 64, 64, None, None, 0, v(16), None, v(16), v(16), None, None)
+    assert st == sv.INVALID_ARG and b"workspace" in L.svdq_last_error_detail()
+    st = L.svdq_quantize_act_dynamic(v(16), 4, 64, 64, None, None, 0, None, v(16), v(16), v(16), None, None)
+    assert st == sv.INVALID_ARG
+    st = L.svdq_quantize_act_dynamic(v(16), 4, 64, 64, None, None, 0, v(16), v(24), v(16), v(16), None, None)
+    assert st == sv.MISALIGNED
+    st = L.svdq_quantize_act_dynamic(v(16), 4, 96, 96, None, None, 0, v(16), v(16), v(16), v(16), None, None)
+    assert st == sv.INVALID_ARG  # K % 64
+
+
 def test_linear_and_awq_validation_is_host_side():
     L = sv.lib()
     v = ctypes.c_void_p
@@ -75,6 +88,20 @@ def test_linear_and_awq_validation_is_host_side():
                                 4, 32, 64, v(16), 32, 2, None)
     assert st == sv.INVALID_ARG  # unknown activation
     assert b"activation=2" in L.svdq_last_error_detail()
+    ys = (v * 3)(v(16), v(16), v(16))
+    st = L.svdq_w4a4_linear_split(v(16), v(16), v(16), None, v(16), v(16), v(16), None, 0, None,
+                                  4, 384, 64, 4, ctypes.cast(ys, v), 128, 0, None)
+    assert st == sv.INVALID_ARG and b"parts=4" in L.svdq_last_error_detail()
+    st = L.svdq_w4a4_linear_split(v(16), v(16), v(16), None, v(16), v(16), v(16), None, 0, None,
+                                  4, 192, 64, 3, ctypes.cast(ys, v), 64, 0, None)
+    assert st == sv.INVALID_ARG and b"multiple of 128" in L.svdq_last_error_detail()
+    ys_null = (v * 3)(v(16), None, v(16))
+    st = L.svdq_w4a4_linear_split(v(16), v(16), v(16), None, v(16), v(16), v(16), None, 0, None,
+                                  4, 384, 64, 3, ctypes.cast(ys_null, v), 128, 0, None)
+    assert st == sv.INVALID_ARG and b"y_parts[1]" in L.svdq_last_error_detail()
+    st = L.svdq_w4a4_linear_split(v(16), v(16), v(16), None, v(16), v(16), v(16), None, 0, None,
+                                  4, 384, 64, 3, ctypes.cast(ys, v), 120, 0, None)
+    assert st == sv.INVALID_ARG  # ldy < N/parts
     st = L.awq_w4a16_linear(v(16), 9, 64, None, v(16), v(16), v(16), 64, None, 32, v(16), None)
     assert st == sv.INVALID_ARG  # M > 8
     st = L.awq_w4a16_linear(v(16), 1, 64, None, v(16), v(16), v(16), 128, None, 32, v(16), None)

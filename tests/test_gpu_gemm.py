@@ -220,3 +220,102 @@ def test_gemm_many_tiles_per_cta(M, K, N, r):
     ref = osv.svdq_linear(q["codes"], q["sf"], q["gs"], xl, cw[cols], sfw[cols], gs_w, L["L2t"][cols],
                           L["bias"][cols])
     assert_gemm_close(y[:, torch.from_numpy(cols).cuda()], ref, f"many tiles M{M} K{K} N{N} r{r}")
+
+
+# ------------------------------------------------ split outputs (fused QKV) --
+def _split_case(M, K, N, r, parts, seed, pad=0):
+    case = workloads.small_case(M, K, N, r, seed=seed)
+    d, L = prepared(case)
+    out = osv.svdq_forward(d["x"], L)
+    w = weights_from_layer(L)
+    lora = f32(out["xl"]) if r else None
+    args = (u8(out["packed"]), u8(out["sf_swizzled"]), f32([out["gs"]]), lora, w)
+    n_part = N // parts
+    ys = None
+    if pad:  # each part a column slice of a wider buffer: ldy = n_part + pad
+        big = [torch.full((M, n_part + pad), 7.0, dtype=torch.bfloat16, device="cuda") for _ in range(parts)]
+        ys = [b[:, :n_part] for b in big]
+    got = sv.w4a4_linear_split(*args, parts=parts, ys=ys)
+    fused = sv.w4a4_linear(*args)
+    torch.cuda.synchronize()
+    if pad:
+        for b in big:  # the padding columns are never written
+            assert (b[:, n_part:].float() == 7.0).all()
+    return got, fused, out["y"]
+
+
+# (M, K, N, r, parts, pad): three parts of 128 (tile width 128 although N
+# is a multiple of 192), three of 384 (192), two of 256 (128), ragged M, a
+# padded leading dimension
+SPLIT = [
+    (200, 512, 384, 32, 3, 0),
+    (256, 512, 1152, 16, 3, 0),
+    (77, 320, 512, 64, 2, 24),
+    (129, 256, 768, 32, 3, 8),
+]
+
+
+@pytest.mark.parametrize("M,K,N,r,parts,pad", SPLIT)
+def test_split_outputs_small(M, K, N, r, parts, pad):
+    got, fused, ref = _split_case(M, K, N, r, parts, seed=M + N + parts, pad=pad)
+    n_part = N // parts
+    # the output bar holds for y, which the parts store side by side (a part's
+    # own rms can be too small a yardstick: on a 129 x 256 part the bf16
+    # rounding of the exact result alone reaches 2.01e-2 of it)
+    assert_gemm_close(torch.cat(got, dim=1), ref, f"parts of M{M} K{K} N{N} r{r}")
+    same_tile = (n_part % 192 == 0) == (N % 192 == 0)
+    for i, y in enumerate(got):
+        cols = slice(i * n_part, (i + 1) * n_part)
+        if same_tile:  # same tiling as the single-output call: the same bits
+            assert torch.equal(y, fused[:, cols]), f"part {i} differs from the single-output call"
+
+
+def test_fused_qkv_split_full_size():
+    # the fused QKV projection: one quantized activation, one GEMM over
+    # [W_q; W_k; W_v], Q, K and V stored in their own [M, 3072] tensors
+    d, L = _full(workloads.QKV[32].name, 32)
+    x = d["x"]
+    gs = osv.act_tensor_scale(x, L["s"])
+    w = weights_from_layer(L)
+    q, sf, lora, gso = sv.quantize_act(bf16(x), w.smooth, w.L1t, f32([gs]))
+    qkv = sv.w4a4_linear_split(q, sf, gso, lora, w, parts=3)
+    fused = sv.w4a4_linear(q, sf, gso, lora, w)
+    torch.cuda.synchronize()
+    n_part = w.N // 3
+    for i in range(3):
+        assert torch.equal(qkv[i], fused[:, i * n_part:(i + 1) * n_part])
+    rows = np.arange(0, x.shape[0], 64)
+    ref = osv.svdq_forward(x[rows], L, gs)["y"]
+    idx = torch.from_numpy(rows).cuda()
+    assert_gemm_close(torch.cat([t[idx] for t in qkv], dim=1), ref, "qkv parts")
+
+
+def test_split_with_gelu_matches_single_output():
+    case = workloads.small_case(256, 512, 1152, 32, seed=77)
+    d, L = prepared(case)
+    out = osv.svdq_forward(d["x"], L)
+    w = weights_from_layer(L)
+    args = (u8(out["packed"]), u8(out["sf_swizzled"]), f32([out["gs"]]), f32(out["xl"]), w)
+    parts = sv.w4a4_linear_split(*args, parts=3, act="gelu")
+    whole = sv.w4a4_linear(*args, act="gelu")
+    torch.cuda.synchronize()
+    assert torch.equal(torch.cat(parts, dim=1), whole)
+
+
+def test_fused_prep_stacks_the_projections():
+    from svdquant_w4a4_gemm_b200 import prep as dprep
+    g = torch.Generator(device="cuda").manual_seed(3)
+    Ws = [(torch.randn(n, 256, device="cuda", generator=g) * 0.02).to(torch.bfloat16) for n in (128, 128, 256)]
+    bs = [torch.randn(128, device="cuda", generator=g).to(torch.bfloat16), None,
+          torch.randn(256, device="cuda", generator=g).to(torch.bfloat16)]
+    xc = torch.randn(64, 256, device="cuda", generator=g).to(torch.bfloat16)
+    # r = 0: no SVD, so the stacked layer must match the concatenation bit for bit
+    fused = dprep.prepare_svdq_fused(Ws, bs, xc, 0)
+    whole = dprep.prepare_svdq(torch.cat(Ws), torch.cat([bs[0], torch.zeros(128, dtype=torch.bfloat16,
+                                                                              device="cuda"), bs[2]]), xc, 0)
+    ranked = dprep.prepare_svdq_fused(Ws, bs, xc, 16)
+    torch.cuda.synchronize()
+    assert fused.N == 512 and ranked.N == 512 and ranked.rank == 16
+    for a, b in ((fused.q_w, whole.q_w), (fused.sf_w, whole.sf_w), (fused.bias, whole.bias),
+                 (fused.smooth, whole.smooth)):
+        assert torch.equal(a, b)

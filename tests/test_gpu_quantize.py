@@ -127,6 +127,61 @@ def test_quantize_repeatable_at_every_ring_depth(M, K, r):
         assert np.linalg.norm(lora0[rows] - xl_ref) <= 1e-4 * np.linalg.norm(xl_ref)
 
 
+# single-pass dynamic scale: the max, a grid barrier and the quantization in
+# one launch.  It must give the same bytes as the max pass + quantize path
+# and the oracle's dynamic scale: small and ragged shapes, one row, several
+# sub-tiles per CTA at every ring depth, and two calls in a row on one
+# workspace (the call clears it).
+@pytest.mark.parametrize("M,K,r,smooth", [(200, 512, 16, True), (1, 128, 128, True), (333, 1024, 0, False),
+                                          (4096, 3072, 32, True), (4608, 3072, 128, True),
+                                          (1000, 12288, 64, True)])
+def test_single_pass_dynamic_scale(M, K, r, smooth):
+    rng = np.random.default_rng(M * 3 + K + r)
+    x = workloads.to_bf16(rng.standard_normal((M, K)).astype(np.float32))
+    x[rng.integers(0, M), rng.integers(0, K)] = 37.5          # one outlier sets the max
+    s = rng.uniform(0.5, 4.0, K).astype(np.float32) if smooth else None
+    L1t = workloads.to_bf16(rng.standard_normal((max(r, 16), K)).astype(np.float32) * 0.05)[:r] if r else None
+    xt = bf16(x)
+    st = None if s is None else f32(s)
+    lt = bf16(L1t) if r else None
+    ws = torch.empty(sv.QUANTIZE_WORKSPACE_BYTES, dtype=torch.uint8, device="cuda")
+    two = [sv.quantize_act_dynamic(xt, st, lt, workspace=ws) for _ in range(2)]
+    base = sv.quantize_act(xt, st, lt, None)
+    torch.cuda.synchronize()
+    sv.check_device_errors()
+    gs_ref = osv.act_tensor_scale(x, s)
+    for q, sf, lora, gs in two:
+        assert gs.item() == gs_ref == base[3].item()
+        assert torch.equal(q, base[0]), "codes: " + describe_byte_mismatch(q.cpu().numpy().ravel(),
+                                                                          base[0].cpu().numpy().ravel())
+        assert torch.equal(sf, base[1])
+        if r:
+            ref = base[2].double()
+            assert (lora.double() - ref).norm() <= 1e-5 * ref.norm()
+    rows = np.arange(0, M, 11)
+    ref = osv.quantize_act(x[rows], s, gs_ref)
+    assert np.array_equal(two[0][0].cpu().numpy()[rows], ref["packed"])
+
+
+def test_single_pass_dynamic_scale_two_workspaces_two_streams():
+    rng = np.random.default_rng(5)
+    xs = [bf16(workloads.to_bf16(rng.standard_normal((2048, 3072)).astype(np.float32) * (1 + i)))
+          for i in range(2)]
+    streams = [torch.cuda.Stream() for _ in range(2)]
+    wss = [torch.zeros(sv.QUANTIZE_WORKSPACE_BYTES, dtype=torch.uint8, device="cuda") for _ in range(2)]
+    outs = [None, None]
+    torch.cuda.synchronize()
+    for i in range(2):
+        with torch.cuda.stream(streams[i]):
+            outs[i] = sv.quantize_act_dynamic(xs[i], None, None, workspace=wss[i])
+    torch.cuda.synchronize()
+    sv.check_device_errors()
+    for i in range(2):
+        base = sv.quantize_act(xs[i], None, None, None)
+        torch.cuda.synchronize()
+        assert torch.equal(outs[i][0], base[0]) and outs[i][3].item() == base[3].item()
+
+
 def test_quantize_strided_rows_and_gs_copy():
     case = workloads.small_case(160, 256, 64, 32, seed=5)
     d, L = prepared(case)

@@ -3,14 +3,16 @@ GEMM's producer never fills one ring slot, so the MMA thread's wait for it
 runs out after the (shortened) limit; every role of the kernel gives up its
 own wait, drains its in-flight copies, frees its tensor memory and returns.
 The host then reads SVDQ_ERR_DEVICE_TIMEOUT, and the context stays usable:
-a normal call right after gives the right answer.  Nothing traps or faults."""
+a normal call right after gives the right answer.  The same for the grid
+barrier of the single-pass dynamic quantize: the first CTA skips its
+arrival and the others' bounded waits run out.  Nothing traps or faults."""
 import numpy as np
 import pytest
 import torch
 
 import workloads
 from oracle import svdq as osv
-from tests._gpu import assert_gemm_close, f32, needs_gpu, prepared, u8, weights_from_layer
+from tests._gpu import assert_gemm_close, bf16, f32, needs_gpu, prepared, u8, weights_from_layer
 
 import svdquant_w4a4_gemm_b200 as sv
 
@@ -38,3 +40,27 @@ def test_gemm_wait_times_out_cleanly_and_context_survives():
     y = sv.w4a4_linear(*args)
     torch.cuda.synchronize()
     assert_gemm_close(y, out["y"], "after a timed-out launch")
+
+
+def test_grid_barrier_wait_times_out_cleanly_and_context_survives():
+    rng = np.random.default_rng(8)
+    x = bf16(workloads.to_bf16(rng.standard_normal((1024, 1024)).astype(np.float32)))
+    L1t = bf16(workloads.to_bf16(rng.standard_normal((32, 1024)).astype(np.float32) * 0.05))
+    sv.check_device_errors()
+    prev_t = sv.set_wait_timeout_ns(50_000_000)   # 50 ms
+    prev_f = sv.lib().svdq_debug_set_fault(2)
+    try:
+        sv.quantize_act_dynamic(x, None, L1t)
+        with pytest.raises(sv.SvdqError) as e:
+            sv.check_device_errors()
+        assert e.value.status == sv.DEVICE_TIMEOUT
+        word = int(str(e.value).split("device error word ")[1].split()[0], 16)
+        assert word & 16, hex(word)                # the grid barrier gave up
+    finally:
+        sv.lib().svdq_debug_set_fault(prev_f)
+        sv.set_wait_timeout_ns(prev_t)
+    sv.check_device_errors()
+    q, sf, lora, gs = sv.quantize_act_dynamic(x, None, L1t)
+    base = sv.quantize_act(x, None, L1t, None)
+    torch.cuda.synchronize()
+    assert torch.equal(q, base[0]) and torch.equal(sf, base[1]) and gs.item() == base[3].item()
