@@ -106,8 +106,12 @@ __device__ __forceinline__ void unit_range(int units, int& u0, int& u1) {
 }
 
 // 14 warps: four of them share some SM sub-partition, whose 16 K registers
-// then allow at most 128 a thread
-__global__ void __maxnreg__(128)
+// then allow at most 128 a thread (checked once per device before the first
+// launch).
+// kSinglePass: the dynamic scale computed in this launch (phase A + grid
+// barrier); a separate instance, so the static path carries none of it.
+template <bool kSinglePass>
+__global__ void __launch_bounds__(kThreads, 1)
     quantize_act_kernel(const __grid_constant__ CUtensorMap tmap_x,
                         const __grid_constant__ CUtensorMap tmap_l1, const QuantParams p) {
   extern __shared__ uint8_t smem_raw[];
@@ -134,7 +138,7 @@ __global__ void __maxnreg__(128)
   unit_range(p.units, u0, u1);
   // ring items: phase A (single-pass dynamic scale only), then phase B
   const int n_units = u1 - u0;
-  const int phase_b0 = p.sync ? n_units : 0;   // first phase-B item
+  const int phase_b0 = kSinglePass ? n_units : 0;   // first phase-B item
   const int n_items = phase_b0 + n_units;
 
   // Warp 0 sets up the barriers and issues the first ns loads right
@@ -189,8 +193,8 @@ __global__ void __maxnreg__(128)
     cta_amax_bits = 0u;
     grid_ok = 1;
   }
-  const float gs = p.sync ? 1.0f : (p.gs_in ? *p.gs_in : tensor_scale_from_amax(*p.amax_src));
-  if (threadIdx.x < 128 && !p.sync) {
+  const float gs = kSinglePass ? 1.0f : (p.gs_in ? *p.gs_in : tensor_scale_from_amax(*p.amax_src));
+  if (threadIdx.x < 128 && !kSinglePass) {
     const float d = e4m3_to_f32(threadIdx.x);
     gs_over_d[threadIdx.x] = (d == 0.0f || threadIdx.x == 127) ? 0.0f : __fdiv_rn(gs, d);
   }
@@ -272,7 +276,7 @@ __global__ void __maxnreg__(128)
     uint32_t ph = 0;
     int i = qw;              // ring item
     float gsq = gs;
-    if (p.sync) {
+    if constexpr (kSinglePass) {
       // phase A: max|x·inv_s| over this warp's sub-tiles; each slot is
       // released as soon as it is read
       bool ok = true;
@@ -336,8 +340,8 @@ __global__ void __maxnreg__(128)
       const bool cta_ok = grid_ok != 0;
       named_bar_sync(1, 32 * kQuantWarps);
       if (!cta_ok) i = n_items;  // the barrier or a wait failed: quantize nothing
-    } else if (p.gs_copy && blockIdx.x == 0 && threadIdx.x == 64) {
-      *p.gs_copy = gs;
+    } else {
+      if (p.gs_copy && blockIdx.x == 0 && threadIdx.x == 64) *p.gs_copy = gs;
     }
     for (; qw < ns && i < n_items; i += ns, ph ^= 1u) {
       const int u = u0 + i - phase_b0;
@@ -566,8 +570,17 @@ svdq_status launch_quantize_act(const LaunchCtx& ctx, const void* x, int64_t M, 
   const size_t smem = quantize_smem_bytes(K, r);
   static bool attr_done[64] = {};
   if (!attr_done[ctx.device & 63]) {
-    cudaFuncSetAttribute(quantize_act_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaFuncSetAttribute(quantize_act_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          static_cast<int>(kSmemLimit));
+    cudaFuncSetAttribute(quantize_act_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         static_cast<int>(kSmemLimit));
+    // four of the 14 warps share one SM sub-partition (16 K registers)
+    cudaFuncAttributes fa{};
+    for (const void* fn : {reinterpret_cast<const void*>(quantize_act_kernel<false>),
+                           reinterpret_cast<const void*>(quantize_act_kernel<true>)})
+      if (cudaFuncGetAttributes(&fa, fn) != cudaSuccess || fa.numRegs > 128)
+        return fail(SVDQ_ERR_CUDA, "quantize_act_kernel uses %d registers a thread; 14 warps allow 128",
+                    fa.numRegs);
     attr_done[ctx.device & 63] = true;
   }
   const int grid = std::min(p.units, ctx.num_sms);
@@ -583,14 +596,14 @@ svdq_status launch_quantize_act(const LaunchCtx& ctx, const void* x, int64_t M, 
     attr[0].val.cooperative = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    const cudaError_t e = cudaLaunchKernelEx(&cfg, quantize_act_kernel, tx, tl, p);
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, quantize_act_kernel<true>, tx, tl, p);
     if (e != cudaSuccess) {
       cudaGetLastError();
       return fail(SVDQ_ERR_CUDA, "quantize_act_kernel (cooperative): %s", cudaGetErrorString(e));
     }
     return SVDQ_OK;
   }
-  quantize_act_kernel<<<grid, kThreads, smem, st>>>(tx, tl, p);
+  quantize_act_kernel<false><<<grid, kThreads, smem, st>>>(tx, tl, p);
   if (svdq_status e = check_launch("quantize_act_kernel")) return e;
   if (!act_gscale) {
     act_scale_finalize_kernel<<<1, 1, 0, st>>>(act_gscale_out);
