@@ -136,6 +136,37 @@ svdq_status svdq_quantize_act_dynamic(const void* x_bf16, int64_t M, int64_t K, 
                                       uint8_t* sf_out, float* lora_out, void* stream);
 
 /*
+ * svdq_quantize_act_dynamic_noalloc — svdq_quantize_act_dynamic for callers
+ * that cannot allocate device memory when they call it: an inference-engine
+ * plugin whose enqueue step must not allocate, a runtime that plans all of
+ * its device memory ahead of time, or a latency-bound path that must not
+ * pay for an allocation.  Such a caller has no workspace to pass, so this
+ * entry point keeps the kernel's scratch (the grid-barrier counter and the
+ * max word, 16 bytes) in a static 256-byte device array inside the library
+ * instead, and allocates nothing (no cudaMalloc, no allocating library call).
+ * The pages have no counterpart; this is an interface convenience.
+ *
+ *   Arguments, outputs and errors as svdq_quantize_act_dynamic, without the
+ *   workspace.  The outputs are those of svdq_quantize_act_dynamic.
+ *   The scratch needed does not depend on M, K or r, so no problem size is
+ *   rejected for it (the array's limit is 256 bytes).
+ *   - The array exists once per device in every process that loads the
+ *     library and is held until the process exits.
+ *   - The first call on a device looks up the array's device address (once
+ *     per device, with that device current); make that first call before
+ *     any stream capture.
+ *   - Every call shares the array and clears it before its kernel runs;
+ *     calls that overlap on the GPU (other streams, other threads) race on
+ *     it and give undefined results.  Serialize them, or use
+ *     svdq_quantize_act_dynamic with a workspace per stream.
+ */
+svdq_status svdq_quantize_act_dynamic_noalloc(const void* x_bf16, int64_t M, int64_t K,
+                                              int64_t ldx, const float* smooth_s,
+                                              const void* L1t_bf16, int r,
+                                              float* act_gscale_out, uint8_t* q_out,
+                                              uint8_t* sf_out, float* lora_out, void* stream);
+
+/*
  * svdq_w4a4_linear — the 4-bit GEMM with the low-rank up-projection fused
  * ("the low-rank up-projection is fused with the 4-bit compute kernel",
  * blog.margrop.com "技术细节 §1" step 4):

@@ -33,6 +33,8 @@ _SIGNATURES = {
     "svdq_quantize_act": (_int, [_vp, _i64, _i64, _i64, _vp, _vp, _int, _vp, _vp, _vp, _vp, _vp, _vp]),
     "svdq_quantize_act_dynamic": (_int, [_vp, _i64, _i64, _i64, _vp, _vp, _int, _vp, _vp, _vp, _vp,
                                          _vp, _vp]),
+    "svdq_quantize_act_dynamic_noalloc": (_int, [_vp, _i64, _i64, _i64, _vp, _vp, _int, _vp, _vp,
+                                                 _vp, _vp, _vp]),
     "svdq_w4a4_linear": (_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _int, _vp,
                                 _i64, _i64, _i64, _vp, _i64, _vp]),
     "svdq_w4a4_linear_act": (_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _int, _vp,

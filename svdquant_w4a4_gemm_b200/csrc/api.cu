@@ -241,6 +241,23 @@ svdq_status svdq_quantize_act_dynamic(const void* x_bf16, int64_t M, int64_t K, 
                         sf_out, lora_out, static_cast<uint32_t*>(workspace), stream);
 }
 
+svdq_status svdq_quantize_act_dynamic_noalloc(const void* x_bf16, int64_t M, int64_t K, int64_t ldx,
+                                              const float* smooth_s, const void* L1t_bf16, int r,
+                                              float* act_gscale_out, uint8_t* q_out,
+                                              uint8_t* sf_out, float* lora_out, void* stream) {
+  if (!act_gscale_out) return fail(SVDQ_ERR_INVALID_ARG, "act_gscale_out must be non-null");
+  LaunchCtx ctx{};
+  if (svdq_status e = device_ctx(stream, &ctx)) return e;
+  // the scratch this call needs (16 bytes) does not grow with M, K or r
+  if (SVDQ_QUANTIZE_WORKSPACE_BYTES > kNoallocScratchBytes)
+    return fail(SVDQ_ERR_INVALID_ARG, "scratch of %d bytes exceeds the %d-byte static array",
+                SVDQ_QUANTIZE_WORKSPACE_BYTES, static_cast<int>(kNoallocScratchBytes));
+  uint32_t* scratch = nullptr;
+  if (svdq_status e = noalloc_quantize_scratch(ctx.device, &scratch)) return e;
+  return quantize_entry(x_bf16, M, K, ldx, smooth_s, L1t_bf16, r, nullptr, act_gscale_out, q_out,
+                        sf_out, lora_out, scratch, stream);
+}
+
 svdq_status svdq_w4a4_linear(const uint8_t* q_act, const uint8_t* sf_act, const float* act_gscale,
                              const float* lora_act, const uint8_t* q_w, const uint8_t* sf_w,
                              const float* w_gscale, const void* L2t_bf16, int r,

@@ -34,6 +34,11 @@ svdq_status check_launch(const char* what);
 // (the API rejects shapes above the 227 KB per-CTA limit before launching).
 size_t quantize_smem_bytes(int64_t K, int r);
 
+// Bytes of the static scratch array behind svdq_quantize_act_dynamic_noalloc,
+// and its device address on `device` (the current device).
+constexpr size_t kNoallocScratchBytes = 256;
+svdq_status noalloc_quantize_scratch(int device, uint32_t** out);
+
 // Kernel launchers (one per translation unit).  Arguments are validated.
 svdq_status launch_quantize_act(const LaunchCtx& ctx, const void* x, int64_t M, int64_t K,
                                 int64_t ldx, const float* smooth_s, const void* L1t, int r,

@@ -56,6 +56,7 @@
 // barrier).  The ring runs through both phases as one sequence of 2n
 // items, item i in slot i mod ns, owned by quantizer warp i mod ns.
 #include <cstdio>
+#include <mutex>
 
 #include "internal.h"
 #include "ptx.cuh"
@@ -514,6 +515,31 @@ int quantize_stages(int64_t K, int r) {
   return std::max(2, std::min(kMaxStages, fit));
 }
 }  // namespace
+
+// Scratch of svdq_quantize_act_dynamic_noalloc: the grid-barrier counter and
+// the max word of the single-pass dynamic scale, in a static device array
+// instead of a caller's workspace.  Every device that loads the library
+// holds it until the process exits; every call shares it.
+static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoallocScratchBytes];
+static_assert(SVDQ_QUANTIZE_WORKSPACE_BYTES <= kNoallocScratchBytes, "the workspace must fit the array");
+
+svdq_status noalloc_quantize_scratch(int device, uint32_t** out) {
+  // its device address, looked up once per device (host code cannot use the
+  // array's name as a device pointer)
+  static std::mutex mu;
+  static void* addr[64] = {};
+  std::lock_guard<std::mutex> lk(mu);
+  if (device < 0 || device >= 64) return fail(SVDQ_ERR_CUDA, "device index %d too large", device);
+  if (!addr[device]) {
+    void* p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess)
+      return fail(SVDQ_ERR_CUDA, "cudaGetSymbolAddress(scratch): %s", cudaGetErrorString(e));
+    addr[device] = p;
+  }
+  *out = static_cast<uint32_t*>(addr[device]);
+  return SVDQ_OK;
+}
 
 size_t quantize_smem_bytes(int64_t K, int r) {
   return quantize_fixed_bytes(K) +

@@ -73,6 +73,8 @@ def test_single_pass_dynamic_quantize_validation_is_host_side():
     assert st == sv.MISALIGNED
     st = L.svdq_quantize_act_dynamic(v(16), 4, 96, 96, None, None, 0, v(16), v(16), v(16), v(16), None, None)
     assert st == sv.INVALID_ARG  # K % 64
+    st = L.svdq_quantize_act_dynamic_noalloc(v(16), 4, 64, 64, None, None, 0, None, v(16), v(16), None, None)
+    assert st == sv.INVALID_ARG and b"act_gscale_out" in L.svdq_last_error_detail()
 
 
 def test_linear_and_awq_validation_is_host_side():
