@@ -3,7 +3,10 @@ linear library.  Argument marshalling only: every step of the layer runs in
 the library's CUDA kernels; torch provides device memory and the stream.
 
     q, sf, lora, gs = quantize_act(x, smooth, L1t, gscale)    # one pass over x
+    q, sf, lora, gs = quantize_act_dynamic(x, smooth, L1t)    # gs_a from x, same launch
     y = w4a4_linear(q, sf, gs, lora, layer)                   # FP4 GEMM + low-rank + bias
+    h = w4a4_linear(q, sf, gs, lora, up_layer, act="gelu")    # ... + GELU(tanh) epilogue
+    q_, k_, v_ = w4a4_linear_split(q, sf, gs, lora, qkv_layer, parts=3)  # fused QKV
     y = awq_w4a16_linear(x, act_scale_inv, qweight, scales, zeros, bias)
 
 The C ABI (include/svdq.h) is also exposed raw as ``lib()`` for callers that

@@ -29,6 +29,11 @@ def test_library_exports_every_declared_function():
         assert hasattr(L, n), n
 
 
+def test_binding_types_every_declared_function():
+    # a ctypes call without argtypes would pass 64-bit pointers and sizes as C ints
+    assert set(_declared_functions()) <= set(sv._SIGNATURES)
+
+
 def test_status_strings_and_version():
     L = sv.lib()
     assert L.svdq_version() >= 100
