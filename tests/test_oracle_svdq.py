@@ -215,6 +215,20 @@ def test_smoothing_factor_definition():
     np.testing.assert_allclose(s, [np.sqrt(2 / 0.5), np.sqrt(8 / 0.02)], rtol=1e-6)
 
 
+def test_smoothing_balances_activation_and_weight_ranges():
+    # the α = 0.5 balance the smoothing is chosen for: after x̂ = x·diag(1/s)
+    # and Ŵ = W·diag(s), every input channel's activation max equals its
+    # weight max (both sqrt(max|x_k| · max|W_k|)), and the product is unchanged
+    rng = _rng(17)
+    x = rng.standard_normal((64, 48)) * rng.uniform(0.1, 30.0, 48)[None, :]
+    W = rng.standard_normal((40, 48)) * rng.uniform(0.001, 0.5, 48)[None, :]
+    s = prep.smoothing_factors(x, W).astype(np.float64)
+    xmax = np.abs(x / s[None, :]).max(axis=0)
+    wmax = np.abs(W * s[None, :]).max(axis=0)
+    np.testing.assert_allclose(xmax, wmax, rtol=1e-6)
+    np.testing.assert_allclose((x / s[None, :]) @ (W * s[None, :]).T, x @ W.T, rtol=1e-10, atol=1e-12)
+
+
 @pytest.mark.parametrize("frac,mult", [(0.01, 20.0), (0.02, 30.0)])
 def test_svd_branch_lowers_error_on_outlier_inputs(frac, mult):
     # the pages' central claim: plain W4A4 is hurt by outliers; SVDQuant's
