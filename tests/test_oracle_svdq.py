@@ -246,3 +246,66 @@ def test_svd_branch_lowers_error_on_outlier_inputs(frac, mult):
     e_plain = np.linalg.norm(svdq.svdq_forward(d["x"], L0)["y"] - exact) / np.linalg.norm(exact)
     assert err[32] < 0.8 * err[0], err
     assert err[32] < e_plain
+
+
+def test_inv_smooth_is_the_correctly_rounded_reciprocal():
+    # 1/s in fp64 is exact enough that one rounding to fp32 gives RN32(1/s):
+    # for a 24-bit s, 1/s is never within 2^-49 of an fp32 midpoint
+    s = _rng(21).uniform(1e-3, 1e3, 200000).astype(np.float32)
+    got = svdq.inv_smooth(s, s.size)
+    want = (1.0 / s.astype(np.float64)).astype(np.float32)
+    assert np.array_equal(got.view(np.uint32), want.view(np.uint32))
+    assert np.array_equal(svdq.inv_smooth(None, 7), np.ones(7, np.float32))
+
+
+def test_act_tensor_scale_puts_the_largest_group_at_448():
+    rng = _rng(22)
+    x = codecs.bf16_round((rng.standard_normal((96, 128)) * 3).astype(np.float32))
+    s = rng.uniform(0.5, 2.0, 128).astype(np.float32)
+    gs = svdq.act_tensor_scale(x, s)
+    q = svdq.quantize_act(x, s, gs)
+    assert codecs.e4m3_decode(q["sf"]).max() == 448.0   # the E4M3 maximum, exactly
+    assert svdq.act_tensor_scale(np.zeros((4, 64), np.float32), None) == 1.0
+
+
+def test_low_rank_factors_meet_the_eckart_young_bound():
+    # any rank-r matrix leaves at least the tail singular energy; the bf16
+    # factors may add at most their own rounding to it
+    rng = _rng(23)
+    N, K, r = 60, 40, 8
+    signal = rng.standard_normal((N, r)) @ rng.standard_normal((r, K))
+    What = signal + 1e-3 * rng.standard_normal((N, K))
+    L1t, L2t = prep.low_rank_factors(What, r)
+    assert L1t.shape == (r, K) and L2t.shape == (N, r)
+    resid = np.linalg.norm(What - L2t.astype(np.float64) @ L1t.astype(np.float64))
+    sig = np.linalg.svd(What, compute_uv=False)
+    tail = np.sqrt(np.sum(sig[r:] ** 2))
+    assert tail * (1 - 1e-12) <= resid <= tail + 8e-3 * np.linalg.norm(What)
+    z1, z2 = prep.low_rank_factors(What, 0)
+    assert z1.shape == (0, K) and z2.shape == (N, 0)
+
+
+def test_svd_of_smoothed_reconstructs_the_transposed_weight():
+    What = _rng(24).standard_normal((30, 20))
+    U, S, Vt = prep.svd_of_smoothed(What)
+    np.testing.assert_allclose((U * S[None, :]) @ Vt, What.T, atol=1e-12)
+    np.testing.assert_allclose(U.T @ U, np.eye(U.shape[1]), atol=1e-12)
+    assert np.all(np.diff(S) <= 0)
+
+
+def test_awq_scales_follow_the_square_root_of_channel_means():
+    rng = _rng(25)
+    x = rng.standard_normal((128, 64)) * rng.uniform(0.01, 10.0, 64)[None, :]
+    a = prep.awq_scales(x)
+    m = np.abs(x).mean(axis=0)
+    ratio = a / np.sqrt(m)
+    np.testing.assert_allclose(ratio, ratio[0], rtol=1e-12)   # a_k ∝ mean|x_k|^(1/2)
+    assert a.max() * a.min() == pytest.approx(1.0, rel=1e-12)
+
+
+def test_bf16_bit_helpers_match_torch():
+    import torch
+    x = (_rng(26).standard_normal(20000) * 100).astype(np.float32)
+    t = torch.from_numpy(x).to(torch.bfloat16)
+    assert np.array_equal(codecs.bf16_bits(x), t.view(torch.int16).numpy().view(np.uint16))
+    assert np.array_equal(codecs.bf16_from_bits(codecs.bf16_bits(x)), t.float().numpy())
