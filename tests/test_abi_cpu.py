@@ -29,6 +29,29 @@ def test_library_exports_every_declared_function():
         assert hasattr(L, n), n
 
 
+def test_every_declared_function_has_its_doc_comment():
+    # the header is the boundary's documentation: each entry point comes right
+    # after the comment that states its operation, layouts, ownership and errors
+    lines = open(os.path.join(ROOT, "include", "svdq.h")).read().splitlines()
+    in_comment, seen = False, set()
+    for i, line in enumerate(lines):
+        if in_comment:
+            in_comment = "*/" not in line
+            continue
+        if line.lstrip().startswith("/*"):
+            in_comment = "*/" not in line
+            continue
+        m = re.match(r"^[A-Za-z_].*?\b((?:svdq|awq)_\w+)\s*\(", line)
+        if not m or line.startswith("#"):
+            continue
+        j = i - 1
+        while j >= 0 and (not lines[j].strip() or lines[j].startswith("#define") or lines[j].startswith("enum")):
+            j -= 1
+        assert lines[j].rstrip().endswith("*/"), f"{m.group(1)} has no doc comment"
+        seen.add(m.group(1))
+    assert set(_declared_functions()) <= seen
+
+
 def test_binding_types_every_declared_function():
     # a ctypes call without argtypes would pass 64-bit pointers and sizes as C ints
     assert set(_declared_functions()) <= set(sv._SIGNATURES)
