@@ -75,12 +75,12 @@ size_t svdq_nvfp4_scale_bytes(int64_t rows, int64_t K);
 /*
  * svdq_quantize_act — smoothing + NVFP4 activation quantization + low-rank
  * down-projection, in one pass over x (the quantize kernel of the pages'
- * fusion: "the low-rank down-projection is fused with the quantization
- * kernel", blog.margrop.com "技术细节 §1" step 4).
+ * fusion: the pages put the low-rank down-projection inside the kernel
+ * that quantizes the activations; blog.margrop.com "技术细节 §1" step 4).
  *
  *   x_bf16      [M, K] bf16, row stride ldx elements (ldx >= K, ldx % 8 == 0).
  *   M, K        M >= 1, K >= 64, K % 64 == 0.
- *   smooth_s    [K] fp32 smoothing vector s (> 0), 8-byte aligned.  The
+ *   smooth_s    [K] fp32 smoothing vector s (> 0), 4-byte aligned.  The
  *               kernel multiplies x by RN_fp32(1/s_k).  NULL = no smoothing.
  *   L1t_bf16    L1ᵀ, [r, K] bf16 row-major (K contiguous).  Ignored if r == 0.
  *   r           low-rank rank: 0 (no branch), 16, 32, 64 or 128.
@@ -167,9 +167,9 @@ svdq_status svdq_quantize_act_dynamic_noalloc(const void* x_bf16, int64_t M, int
                                               uint8_t* sf_out, float* lora_out, void* stream);
 
 /*
- * svdq_w4a4_linear — the 4-bit GEMM with the low-rank up-projection fused
- * ("the low-rank up-projection is fused with the 4-bit compute kernel",
- * blog.margrop.com "技术细节 §1" step 4):
+ * svdq_w4a4_linear — the 4-bit GEMM with the low-rank up-projection done
+ * inside the same kernel, so the 16-bit branch adds no pass over memory
+ * (blog.margrop.com "技术细节 §1", SVDQuant step 4):
  *
  *   y = bf16( dec(A)·dec(W)ᵀ + lora_act·L2 + bias )
  *

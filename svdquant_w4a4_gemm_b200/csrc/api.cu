@@ -12,6 +12,8 @@
 #include <cstdlib>
 #include <cstring>
 #include <mutex>
+#include <utility>
+#include <vector>
 
 #include "internal.h"
 #include "ptx.cuh"
@@ -25,10 +27,17 @@ namespace {
 
 thread_local char t_detail[512] = "";
 
+// Per device.  Addresses of __device__ symbols and kernel attributes belong
+// to a CUDA context: after a device reset the runtime creates a new primary
+// context, so they are looked up again whenever the current context's ID
+// (unique for the life of the process) differs from the one they were
+// taken in.
 struct DeviceInfo {
   bool init = false;
   int major = 0, minor = 0, num_sms = 0;
+  unsigned long long ctx_id = 0;                  // context of err_word and attrs
   uint32_t* err_word = nullptr;
+  std::vector<std::pair<const void*, int>> attrs;  // (kernel, dynamic smem bytes) opted in
   cudaError_t init_err = cudaSuccess;
 };
 
@@ -43,6 +52,29 @@ using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t
                                    const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
                                    CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 EncodeTiledFn g_encode = nullptr;
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long*);
+CtxGetCurrentFn g_ctx_current = nullptr;
+CtxGetIdFn g_ctx_id = nullptr;
+
+template <typename Fn>
+cudaError_t driver_fn(const char* name, Fn* out) {
+  void* fn = nullptr;
+  cudaDriverEntryPointQueryResult q{};
+  cudaError_t e = cudaGetDriverEntryPoint(name, &fn, cudaEnableDefault, &q);
+  if (e == cudaSuccess && q != cudaDriverEntryPointSuccess) e = cudaErrorSymbolNotFound;
+  if (e == cudaSuccess) *out = reinterpret_cast<Fn>(fn);
+  return e;
+}
+
+// ID of the calling thread's current context (0 if none is current).
+unsigned long long current_ctx_id() {
+  CUcontext c = nullptr;
+  unsigned long long id = 0;
+  if (g_ctx_current(&c) != CUDA_SUCCESS || !c) return 0;
+  if (g_ctx_id(c, &id) != CUDA_SUCCESS) return 0;
+  return id;
+}
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -71,28 +103,15 @@ svdq_status device_ctx(void* stream, LaunchCtx* ctx) {
     return fail(SVDQ_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
   if (dev < 0 || dev >= kMaxDevices) return fail(SVDQ_ERR_CUDA, "device index %d too large", dev);
   DeviceInfo& d = g_dev[dev];
-  {
-    std::lock_guard<std::mutex> lk(g_mu);
-    if (!d.init) {
-      cudaDeviceGetAttribute(&d.major, cudaDevAttrComputeCapabilityMajor, dev);
-      cudaDeviceGetAttribute(&d.minor, cudaDevAttrComputeCapabilityMinor, dev);
-      cudaDeviceGetAttribute(&d.num_sms, cudaDevAttrMultiProcessorCount, dev);
-      if (d.major == 10 && d.minor == 0) {
-        void* p = nullptr;
-        d.init_err = cudaGetSymbolAddress(&p, g_err_word);
-        d.err_word = static_cast<uint32_t*>(p);  // zero since the module loaded
-      }
-      if (!g_encode && d.init_err == cudaSuccess) {
-        void* fn = nullptr;
-        cudaDriverEntryPointQueryResult q{};
-        d.init_err = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q);
-        if (d.init_err == cudaSuccess && q == cudaDriverEntryPointSuccess)
-          g_encode = reinterpret_cast<EncodeTiledFn>(fn);
-        else if (d.init_err == cudaSuccess)
-          d.init_err = cudaErrorSymbolNotFound;
-      }
-      d.init = true;
-    }
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (!d.init) {
+    cudaDeviceGetAttribute(&d.major, cudaDevAttrComputeCapabilityMajor, dev);
+    cudaDeviceGetAttribute(&d.minor, cudaDevAttrComputeCapabilityMinor, dev);
+    cudaDeviceGetAttribute(&d.num_sms, cudaDevAttrMultiProcessorCount, dev);
+    if (!g_encode) d.init_err = driver_fn("cuTensorMapEncodeTiled", &g_encode);
+    if (!g_ctx_current && d.init_err == cudaSuccess) d.init_err = driver_fn("cuCtxGetCurrent", &g_ctx_current);
+    if (!g_ctx_id && d.init_err == cudaSuccess) d.init_err = driver_fn("cuCtxGetId", &g_ctx_id);
+    d.init = true;
   }
   if (!(d.major == 10 && d.minor == 0))
     return fail(SVDQ_ERR_UNSUPPORTED_DEVICE,
@@ -101,8 +120,22 @@ svdq_status device_ctx(void* stream, LaunchCtx* ctx) {
                 dev, d.major, d.minor);
   if (d.init_err != cudaSuccess)
     return fail(SVDQ_ERR_CUDA, "device setup: %s", cudaGetErrorString(d.init_err));
+  unsigned long long id = current_ctx_id();
+  if (id == 0 || id != d.ctx_id) {
+    // first call in this context (the symbol lookup also makes the
+    // device's primary context current if none was)
+    void* p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_err_word);
+    if (e != cudaSuccess) return fail(SVDQ_ERR_CUDA, "cudaGetSymbolAddress(error word): %s", cudaGetErrorString(e));
+    id = current_ctx_id();
+    if (id == 0) return fail(SVDQ_ERR_CUDA, "no current CUDA context on device %d", dev);
+    d.err_word = static_cast<uint32_t*>(p);  // zero since the module loaded in this context
+    d.attrs.clear();
+    d.ctx_id = id;
+  }
   ctx->stream = static_cast<cudaStream_t>(stream);
   ctx->device = dev;
+  ctx->ctx_id = id;
   ctx->num_sms = d.num_sms;
   ctx->err_word = d.err_word;
   ctx->timeout_ns = g_timeout_ns;
@@ -125,6 +158,27 @@ svdq_status fail(svdq_status st, const char* fmt, ...) {
   std::vsnprintf(t_detail, sizeof(t_detail), fmt, ap);
   va_end(ap);
   return st;
+}
+
+svdq_status set_smem_attr(const LaunchCtx& ctx, const void* kernel, int bytes) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  DeviceInfo& d = g_dev[ctx.device];
+  if (d.ctx_id != ctx.ctx_id) d.attrs.clear();  // another context since the call began
+  for (const auto& a : d.attrs)
+    if (a.first == kernel && a.second >= bytes) return SVDQ_OK;
+  const cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return fail(SVDQ_ERR_CUDA, "cudaFuncSetAttribute(%d bytes of shared memory): %s", bytes,
+                cudaGetErrorString(e));
+  }
+  for (auto& a : d.attrs)
+    if (a.first == kernel) {
+      a.second = bytes;
+      return SVDQ_OK;
+    }
+  d.attrs.emplace_back(kernel, bytes);
+  return SVDQ_OK;
 }
 
 svdq_status check_launch(const char* what) {
@@ -253,7 +307,7 @@ svdq_status svdq_quantize_act_dynamic_noalloc(const void* x_bf16, int64_t M, int
     return fail(SVDQ_ERR_INVALID_ARG, "scratch of %d bytes exceeds the %d-byte static array",
                 SVDQ_QUANTIZE_WORKSPACE_BYTES, static_cast<int>(kNoallocScratchBytes));
   uint32_t* scratch = nullptr;
-  if (svdq_status e = noalloc_quantize_scratch(ctx.device, &scratch)) return e;
+  if (svdq_status e = noalloc_quantize_scratch(ctx, &scratch)) return e;
   return quantize_entry(x_bf16, M, K, ldx, smooth_s, L1t_bf16, r, nullptr, act_gscale_out, q_out,
                         sf_out, lora_out, scratch, stream);
 }

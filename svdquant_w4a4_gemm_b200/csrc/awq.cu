@@ -265,13 +265,8 @@ svdq_status launch_awq_w4a16(const LaunchCtx& ctx, const void* x, int64_t M, int
   const int nt = M <= 4 ? 1 : 2;
   const size_t smem = static_cast<size_t>(K) * 16 * nt +
                       static_cast<size_t>(kSplit - 1) * kTilesPerCta * 32 * 4 * nt * sizeof(float);
-  static bool attr_done[2][64] = {};
-  if (!attr_done[nt - 1][ctx.device & 63]) {
-    cudaFuncSetAttribute(nt == 1 ? awq_w4a16_kernel<1> : awq_w4a16_kernel<2>,
-                         cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
-    attr_done[nt - 1][ctx.device & 63] = true;
-  }
   auto kern = nt == 1 ? awq_w4a16_kernel<1> : awq_w4a16_kernel<2>;
+  if (svdq_status e = set_smem_attr(ctx, reinterpret_cast<const void*>(kern), 227 * 1024)) return e;
   kern<<<grid, kThreads, smem, ctx.stream>>>(
       static_cast<const uint16_t*>(x), static_cast<int>(M), static_cast<int>(K), act_scale_inv,
       qweight, static_cast<const __half*>(scales), static_cast<const __half*>(zeros),

@@ -1,6 +1,7 @@
 // gemm.cu — svdq_w4a4_linear: the NVFP4 W4A4 GEMM with the low-rank
-// up-projection fused in ("the low-rank up-projection is fused with the
-// 4-bit compute kernel", blog.margrop.com "技术细节 §1", SVDQuant step 4).
+// up-projection computed in the same kernel, into the same accumulator
+// (blog.margrop.com "技术细节 §1", SVDQuant step 4: the pages pair the
+// branch's up-projection with the 4-bit GEMM so it costs no extra pass).
 //
 //   y = bf16( α·acc + bias ),  α = 1/(gs_a·gs_w)
 //   acc = Σ_k e2m1_a·sfa · e2m1_w·sfw      (kind::mxf4nvf4 block-scaled MMAs)
@@ -575,12 +576,9 @@ svdq_status launch_bn(const LaunchCtx& ctx, const CUtensorMap& ta, const CUtenso
   using L = Layout<BN>;
   const size_t smem = 1024 + static_cast<size_t>(L::kRing) + kEpiWarps * L::kBoxBytes + L::kBias +
                       8 * (4 * kStages + 2 * kMaxRegions + 4) + 16;
-  static bool attr_done[64] = {};
-  if (!attr_done[ctx.device & 63]) {
-    cudaFuncSetAttribute(w4a4_gemm_kernel<BN, ACT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         static_cast<int>(smem));
-    attr_done[ctx.device & 63] = true;
-  }
+  if (svdq_status e = set_smem_attr(ctx, reinterpret_cast<const void*>(w4a4_gemm_kernel<BN, ACT>),
+                                    static_cast<int>(smem)))
+    return e;
   p.tiles_n = (p.N + BN - 1) / BN;
   p.tiles = p.tiles_n * ((p.M + kBM - 1) / kBM);
   const int grid = std::min(p.tiles, ctx.num_sms);

@@ -13,6 +13,7 @@ namespace svdq {
 struct LaunchCtx {
   cudaStream_t stream;
   int device;
+  unsigned long long ctx_id;  // current CUDA context (its process-unique ID)
   int num_sms;
   uint32_t* err_word;    // device error word of `device`
   uint64_t timeout_ns;   // bound on every in-kernel wait
@@ -30,14 +31,18 @@ bool make_tmap_2d(CUtensorMap* map, const void* base, CUtensorMapDataType dtype,
 svdq_status fail(svdq_status st, const char* fmt, ...);
 svdq_status check_launch(const char* what);
 
+// Opt `kernel` in to `bytes` of dynamic shared memory in the current context
+// (once per context and kernel; thread-safe).  SVDQ_ERR_CUDA if refused.
+svdq_status set_smem_attr(const LaunchCtx& ctx, const void* kernel, int bytes);
+
 // Shared memory the quantize kernel needs for a [*, K] activation at rank r
 // (the API rejects shapes above the 227 KB per-CTA limit before launching).
 size_t quantize_smem_bytes(int64_t K, int r);
 
 // Bytes of the static scratch array behind svdq_quantize_act_dynamic_noalloc,
-// and its device address on `device` (the current device).
+// and its device address in the current context of ctx.device.
 constexpr size_t kNoallocScratchBytes = 256;
-svdq_status noalloc_quantize_scratch(int device, uint32_t** out);
+svdq_status noalloc_quantize_scratch(const LaunchCtx& ctx, uint32_t** out);
 
 // Kernel launchers (one per translation unit).  Arguments are validated.
 svdq_status launch_quantize_act(const LaunchCtx& ctx, const void* x, int64_t M, int64_t K,

@@ -523,19 +523,24 @@ int quantize_stages(int64_t K, int r) {
 static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoallocScratchBytes];
 static_assert(SVDQ_QUANTIZE_WORKSPACE_BYTES <= kNoallocScratchBytes, "the workspace must fit the array");
 
-svdq_status noalloc_quantize_scratch(int device, uint32_t** out) {
-  // its device address, looked up once per device (host code cannot use the
-  // array's name as a device pointer)
+svdq_status noalloc_quantize_scratch(const LaunchCtx& ctx, uint32_t** out) {
+  // its device address, looked up once per device and context with that
+  // device current (host code cannot use the array's name as a device
+  // pointer; a device reset makes a new context, where the array has a new
+  // address)
   static std::mutex mu;
   static void* addr[64] = {};
+  static unsigned long long ctx_of[64] = {};
   std::lock_guard<std::mutex> lk(mu);
+  const int device = ctx.device;
   if (device < 0 || device >= 64) return fail(SVDQ_ERR_CUDA, "device index %d too large", device);
-  if (!addr[device]) {
+  if (!addr[device] || ctx_of[device] != ctx.ctx_id) {
     void* p = nullptr;
     const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
     if (e != cudaSuccess)
       return fail(SVDQ_ERR_CUDA, "cudaGetSymbolAddress(scratch): %s", cudaGetErrorString(e));
     addr[device] = p;
+    ctx_of[device] = ctx.ctx_id;
   }
   *out = static_cast<uint32_t*>(addr[device]);
   return SVDQ_OK;
@@ -594,20 +599,19 @@ svdq_status launch_quantize_act(const LaunchCtx& ctx, const void* x, int64_t M, 
     if (svdq_status e = check_launch("act_amax_kernel")) return e;
   }
   const size_t smem = quantize_smem_bytes(K, r);
-  static bool attr_done[64] = {};
-  if (!attr_done[ctx.device & 63]) {
-    cudaFuncSetAttribute(quantize_act_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         static_cast<int>(kSmemLimit));
-    cudaFuncSetAttribute(quantize_act_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         static_cast<int>(kSmemLimit));
+  {
     // four of the 14 warps share one SM sub-partition (16 K registers)
-    cudaFuncAttributes fa{};
-    for (const void* fn : {reinterpret_cast<const void*>(quantize_act_kernel<false>),
-                           reinterpret_cast<const void*>(quantize_act_kernel<true>)})
-      if (cudaFuncGetAttributes(&fa, fn) != cudaSuccess || fa.numRegs > 128)
-        return fail(SVDQ_ERR_CUDA, "quantize_act_kernel uses %d registers a thread; 14 warps allow 128",
-                    fa.numRegs);
-    attr_done[ctx.device & 63] = true;
+    static const bool regs_ok = [] {
+      cudaFuncAttributes fa{};
+      for (const void* fn : {reinterpret_cast<const void*>(quantize_act_kernel<false>),
+                             reinterpret_cast<const void*>(quantize_act_kernel<true>)})
+        if (cudaFuncGetAttributes(&fa, fn) != cudaSuccess || fa.numRegs > 128) return false;
+      return true;
+    }();
+    if (!regs_ok) return fail(SVDQ_ERR_CUDA, "quantize_act_kernel needs more than 128 registers a thread");
+    const void* fn = single_pass ? reinterpret_cast<const void*>(quantize_act_kernel<true>)
+                                 : reinterpret_cast<const void*>(quantize_act_kernel<false>);
+    if (svdq_status e = set_smem_attr(ctx, fn, static_cast<int>(kSmemLimit))) return e;
   }
   const int grid = std::min(p.units, ctx.num_sms);
   if (single_pass) {

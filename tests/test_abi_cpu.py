@@ -86,8 +86,19 @@ def test_quantize_validation_is_host_side():
     assert _q(r=24) == sv.INVALID_ARG
     assert _q(r=32) == sv.INVALID_ARG          # needs L1t and lora
     assert _q(gs=None) == sv.INVALID_ARG       # dynamic needs gs_out
+    assert _q(K=96) == sv.INVALID_ARG
+    assert b"K=96" in sv.lib().svdq_last_error_detail()
     assert _q(x=24) == sv.MISALIGNED
-    assert b"K=96" in sv.lib().svdq_last_error_detail() or True
+    assert b"aligned" in sv.lib().svdq_last_error_detail()
+    assert _q(s=18) == sv.MISALIGNED           # smooth_s: 4-byte alignment, as the header states
+
+
+def test_smooth_s_needs_only_4_byte_alignment(monkeypatch):
+    # a forced unsupported capability stops the call at the device check,
+    # after validation and before any launch, on any machine
+    monkeypatch.setenv("SVDQ_TEST_FORCE_CC", "9.0")
+    assert _q(s=20) == sv.UNSUPPORTED_DEVICE
+    assert _q(s=18) == sv.MISALIGNED
 
 
 def test_single_pass_dynamic_quantize_validation_is_host_side():
