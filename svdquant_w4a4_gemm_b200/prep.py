@@ -4,7 +4,11 @@ the low-rank branch, quantize the residual; blog.margrop.com "5. 自己量化一
 模型"; keryc.com "Cuantizando tus propios modelos").  Not on the hot path.
 
 * smoothing s_k = sqrt(max_m|x_cal[m,k]| / max_n|W[n,k]|) (clamped >= 1e-5);
-* truncated SVD of Ŵ = W·diag(s) (fp32 on the device), Σ split evenly:
+* rank-r truncated SVD of Ŵ = W·diag(s) (fp32 on the device) by a
+  randomized range finder (Halko, Martinsson and Tropp 2011, "Finding
+  structure with randomness", Algorithms 4.4 and 5.1: a seeded Gaussian
+  sketch with oversampling, a few power iterations re-orthonormalized by QR,
+  then the SVD of the small projected matrix); Σ split evenly:
   L1 = U_r·√Σ, L2 = √Σ·V_rᵀ, stored bf16 as L1ᵀ [r, K] and L2ᵀ [N, r];
 * residual R = Ŵ − L2ᵀ·L1ᵀ, gs_w = 2688 / max|R|, and R is NVFP4-quantized
   by this library's own ``svdq_quantize_act`` (R rounded to bf16 first);
@@ -14,6 +18,30 @@ the low-rank branch, quantize the residual; blog.margrop.com "5. 自己量化一
 import torch
 
 from . import SvdqWeights, quantize_act
+
+
+def randomized_svd(A, r, oversample=16, power_iters=4, seed=0):
+    """Top-r singular triplets of A [K, N] (fp32): (U [K, r], S [r], Vh [r, N]).
+
+    Sketch Y = A·Ω with Ω [N, r + p] Gaussian (seeded, so the prep is
+    repeatable), q power iterations Y ← A·(Aᵀ·Y) with a QR after each
+    product (keeps the small singular directions from drowning in
+    round-off), Q = qr(Y), then the exact SVD of B = Qᵀ·A [(r + p), N] and
+    U = Q·U_B.  The range error shrinks like (σ_{r+p+1}/σ_r)^(2q+1), so a
+    spectrum with a clear gap after the outlier directions is found to fp32
+    accuracy, and a flat tail to a residual within a fraction of a percent of
+    the Eckart-Young optimum."""
+    K, N = A.shape
+    k = min(r + oversample, K, N)
+    g = torch.Generator(device=A.device)
+    g.manual_seed(seed)
+    omega = torch.randn(N, k, generator=g, device=A.device, dtype=A.dtype)
+    Q, _ = torch.linalg.qr(A @ omega)
+    for _ in range(power_iters):
+        Z, _ = torch.linalg.qr(A.T @ Q)
+        Q, _ = torch.linalg.qr(A @ Z)
+    Ub, S, Vh = torch.linalg.svd(Q.T @ A, full_matrices=False)
+    return (Q @ Ub)[:, :r], S[:r], Vh[:r, :]
 
 
 def prepare_svdq(W, bias, x_cal, r, smooth=True):
@@ -28,7 +56,7 @@ def prepare_svdq(W, bias, x_cal, r, smooth=True):
         s = (xmax / wmax).sqrt()
     What = Wf * (s[None, :] if s is not None else 1.0)
     if r > 0:
-        U, S, Vh = torch.linalg.svd(What.T, full_matrices=False)
+        U, S, Vh = randomized_svd(What.T.contiguous(), r)
         root = S[:r].sqrt()
         L1t = (U[:, :r] * root[None, :]).T.contiguous().to(torch.bfloat16)
         L2t = (root[:, None] * Vh[:r, :]).T.contiguous().to(torch.bfloat16)

@@ -1,12 +1,18 @@
 """The library's on-device weight preparation (prep.py) against the oracle's
 CPU preparation.
 
-The two cannot agree bit for bit: the device takes the SVD in fp32 (the
-oracle in fp64), rounds the residual to bf16 before quantizing it with the
-library's own quantize call, and reduces the AWQ channel means in another
-order.  So the device prep is held to what it must deliver:
+The two cannot agree bit for bit: the device takes a randomized SVD in fp32
+(the oracle the exact one in fp64), rounds the residual to bf16 before
+quantizing it with the library's own quantize call, and reduces the AWQ
+channel means in another order.  A randomized SVD does not return the exact
+top-r factors where the spectrum has no gap (the Gaussian bulk behind the
+outlier directions): any r directions of a flat tail are equally good.  So
+the device prep is held to what it must deliver:
 - smoothing factors equal to the oracle's within fp32 rounding;
-- the same rank-r branch (the product L2ᵀ·L1ᵀ within bf16 rounding);
+- a rank-r branch as good as the exact truncated SVD: its residual
+  ||Ŵ − L2ᵀ·L1ᵀ||_F within 1 % of the oracle's (Eckart-Young optimal up
+  to the bf16 rounding of the factors), and the same leading singular
+  values (the outlier directions, which do have a gap) within 1 %;
 - a layer as good as the oracle-prepared one: run through the same kernels,
   its error against the exact fp64 linear x·Wᵀ + b is within 10 % (+1e-3)
   of the oracle-prepared layer's error;
@@ -47,9 +53,16 @@ def test_device_svdq_prep_is_as_good_as_the_oracle_prep(case):
     sv.check_device_errors()
     s_dev = wd.smooth.cpu().numpy().astype(np.float64)
     assert np.abs(s_dev / Lo["s"].astype(np.float64) - 1).max() <= 1e-6
-    P_dev = (wd.L2t.float() @ wd.L1t.float()).cpu().numpy()
+    P_dev = (wd.L2t.float() @ wd.L1t.float()).cpu().numpy().astype(np.float64)
     P_orc = Lo["L2t"].astype(np.float64) @ Lo["L1t"].astype(np.float64)
-    assert _rel(P_dev, P_orc) <= 1e-2
+    What = np.asarray(d["W"], np.float64) * Lo["s"].astype(np.float64)[None, :]
+    res_dev = np.linalg.norm(What - P_dev)
+    res_orc = np.linalg.norm(What - P_orc)
+    assert res_dev <= 1.01 * res_orc, (res_dev, res_orc)
+    n_out = len(workloads.outlier_channels(case.K, case.outlier_frac, case.seed))
+    sv_dev = np.linalg.svd(P_dev, compute_uv=False)[:n_out]
+    sv_orc = np.linalg.svd(P_orc, compute_uv=False)[:n_out]
+    assert np.abs(sv_dev / sv_orc - 1).max() <= 1e-2, (sv_dev, sv_orc)
     y_exact = d["x"].astype(np.float64) @ np.asarray(d["W"], np.float64).T + np.asarray(d["bias"], np.float64)
     e_dev = _rel(y_dev.float().cpu().numpy(), y_exact)
     e_orc = _rel(y_orc.float().cpu().numpy(), y_exact)

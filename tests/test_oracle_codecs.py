@@ -134,6 +134,20 @@ def test_scale_layout_is_a_bijection_onto_padded_blocks(rows_, cols):
         assert o[0, 4] - o[0, 0] == 512
 
 
+def test_scale_layout_matches_documented_offsets():
+    """Hand-worked byte offsets from the cuBLASLt description of the 1x16
+    block-scale layout (tests/golden/nvfp4_scale_layout.txt): they single out
+    the order of rows inside a 16-byte line (row % 32 picks the line, row //
+    32 the 4-byte word), the order of tiles (scale columns first) and the
+    padding of ragged shapes, which a bijection check cannot tell apart."""
+    pts = rows("nvfp4_scale_layout.txt")
+    assert len(pts) >= 15
+    for n_rows, n_cols, r, c, off in pts:
+        got = int(codecs.scale_offset(int(r), int(c), int(n_cols)))
+        assert got == int(off), (n_rows, n_cols, r, c, got, off)
+        assert got < codecs.scale_buffer_bytes(int(n_rows), int(n_cols))
+
+
 def test_swizzle_round_trip_and_zero_padding():
     sf = np.random.default_rng(2).integers(1, 255, (130, 12)).astype(np.uint8)
     buf = codecs.swizzle_scales(sf)
