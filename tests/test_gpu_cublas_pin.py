@@ -37,26 +37,28 @@ def _scale_view(buf, rows, K):
 
 
 def cublas_nvfp4(qa, sfa, qw, sfw, M, N, K):
-    """e2m1(A)·dec(sfa) · (e2m1(W)·dec(sfw))ᵀ by cuBLASLt, bf16 [M, N] (no
-    tensor scales).  Tries torch's scaled_mm API, then the older
-    ``_scaled_mm`` form; returns (y, which)."""
+    """e2m1(A)·dec(sfa) · (e2m1(W)·dec(sfw))ᵀ by cuBLASLt, [M, N] (no tensor
+    scales), in fp32 if cuBLASLt writes fp32 for this kind, else bf16.
+    Tries torch's scaled_mm API, then the older ``_scaled_mm`` form; returns
+    (y, which)."""
     a = qa.view(torch.float4_e2m1fn_x2)
     b = qw.view(torch.float4_e2m1fn_x2).t()          # [K/2, N], column-major
     sa, sb = _scale_view(sfa, M, K), _scale_view(sfw, N, K)
     errors = []
-    try:
-        F = torch.nn.functional
-        y = F.scaled_mm(a, b, sa, F.ScalingType.BlockWise1x16, sb, F.ScalingType.BlockWise1x16,
-                        swizzle_a=F.SwizzleType.SWIZZLE_32_4_4, swizzle_b=F.SwizzleType.SWIZZLE_32_4_4,
-                        output_dtype=torch.bfloat16)
-        return y, "F.scaled_mm"
-    except Exception as e:  # noqa: BLE001 - report every attempt if none works
-        errors.append(f"F.scaled_mm: {e}")
-    try:
-        y = torch._scaled_mm(a, b, sa, sb, out_dtype=torch.bfloat16)
-        return y, "torch._scaled_mm"
-    except Exception as e:  # noqa: BLE001
-        errors.append(f"torch._scaled_mm: {e}")
+    F = torch.nn.functional
+    for dt in (torch.float32, torch.bfloat16):
+        try:
+            y = F.scaled_mm(a, b, sa, F.ScalingType.BlockWise1x16, sb, F.ScalingType.BlockWise1x16,
+                            swizzle_a=F.SwizzleType.SWIZZLE_32_4_4, swizzle_b=F.SwizzleType.SWIZZLE_32_4_4,
+                            output_dtype=dt)
+            return y, f"F.scaled_mm -> {dt}"
+        except Exception as e:  # noqa: BLE001 - report every attempt if none works
+            errors.append(f"F.scaled_mm {dt}: {e}")
+        try:
+            y = torch._scaled_mm(a, b, sa, sb, out_dtype=dt)
+            return y, f"torch._scaled_mm -> {dt}"
+        except Exception as e:  # noqa: BLE001
+            errors.append(f"torch._scaled_mm {dt}: {e}")
     pytest.fail("no cuBLASLt NVFP4 entry in this torch: " + " | ".join(s[:300] for s in errors))
 
 
@@ -83,7 +85,12 @@ def test_oracle_bytes_read_by_cublaslt_give_the_oracle_product(case):
 def test_library_gemm_matches_cublaslt_on_the_quantize_kernels_bytes(case):
     """The quantize kernel's codes and scales with the oracle's weight bytes:
     the library's W4A4 GEMM at r = 0 without bias equals cuBLASLt's result
-    times α = 1/(gs_a·gs_w), within the output bar."""
+    times α = 1/(gs_a·gs_w).  Both sum the same exact products in fp32, so
+    they differ by the output roundings: the library's bf16(α·acc) is within
+    2^-9·|y| of α·acc, and a bf16 cuBLASLt output adds another 2^-9·|y|
+    before α is applied; the accumulation order adds ~1e-6 relative.  Each
+    element is held to that bound (plus 1e-4·rms for the order), and the
+    whole to the relative Frobenius bar."""
     d = workloads.draw_svdq(case)
     L = prep.prepare_svdq_layer(d["x_cal"], d["W"], None, 0)
     w = weights_from_layer(L)
@@ -94,6 +101,13 @@ def test_library_gemm_matches_cublaslt_on_the_quantize_kernels_bytes(case):
     y_cb, which = cublas_nvfp4(qa, sfa, w.q_w, w.sf_w, M, N, K)
     alpha = 1.0 / (np.float64(gs_a) * np.float64(L["gs_w"]))
     ref = y_cb.double().cpu().numpy() * alpha
-    assert_gemm_close(y_lib, ref, f"library GEMM vs cuBLASLt ({which})")
+    y = y_lib.double().cpu().numpy()
+    rounding = 2.0 ** -9 if y_cb.dtype == torch.float32 else 2.0 ** -8
+    rms = np.sqrt(np.mean(ref ** 2))
+    excess = np.abs(y - ref) - (rounding * np.abs(ref) + 1e-4 * rms)
+    assert excess.max() <= 0, f"library GEMM vs cuBLASLt ({which}): {int((excess > 0).sum())} elements " \
+                              f"beyond the rounding bound, worst by {excess.max() / rms:.3e}·rms"
+    rel_f = np.linalg.norm(y - ref) / np.linalg.norm(ref)
+    assert rel_f <= 5e-3, (which, rel_f)
     torch.cuda.synchronize()
     sv.check_device_errors()
