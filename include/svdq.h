@@ -294,6 +294,21 @@ svdq_status svdq_check_device_errors(void* stream);
 uint64_t svdq_set_wait_timeout_ns(uint64_t ns);
 
 /*
+ * svdq_set_gemm_pairs — how later svdq_w4a4_linear* launches from this
+ * process tile the output.  enable = 0 (the default): 128 x 192 tiles where
+ * 192 divides N / parts, else 128 x 128, each on one SM.  enable = 1: where
+ * M > 128, 256 x 192 (or 256 x 128) tiles, each computed by a pair of SMs (a
+ * 2-CTA cluster) with one tcgen05 MMA over both SMs' shared and tensor
+ * memory.  Both give results within the same bound of the exact product (the
+ * accumulation order inside a tile may differ).  On B200 the one-SM tiles
+ * are the faster of the two for the shapes measured (the pair's block scales
+ * are staged into each SM's tensor memory by that SM's warps, and the signal
+ * that both SMs' scales are in place crosses SMs every K step).  Returns the
+ * previous setting.  Host-only; never fails.
+ */
+int svdq_set_gemm_pairs(int enable);
+
+/*
  * svdq_debug_set_fault — TEST HOOK.  flags = 1 makes the next launches of
  * svdq_w4a4_linear skip one producer arrive so that the consumer's bounded
  * wait runs out; flags = 2 makes the first CTA of the next

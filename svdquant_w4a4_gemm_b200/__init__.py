@@ -47,6 +47,7 @@ _SIGNATURES = {
     "awq_w4a16_linear": (_int, [_vp, _i64, _i64, _vp, _vp, _vp, _vp, _int, _vp, _i64, _vp, _vp]),
     "svdq_check_device_errors": (_int, [_vp]),
     "svdq_set_wait_timeout_ns": (_u64, [_u64]),
+    "svdq_set_gemm_pairs": (_int, [_int]),
     "svdq_debug_set_fault": (_int, [_int]),
 }
 
@@ -97,6 +98,13 @@ def check_device_errors(device=None):
 
 def set_wait_timeout_ns(ns):
     return int(lib().svdq_set_wait_timeout_ns(ns))
+
+
+def set_gemm_pairs(enable):
+    """SM-pair (2-CTA, 256-row) tiles for the W4A4 GEMM where the shape allows
+    (default off: one-SM tiles measured faster on B200); returns the previous
+    setting."""
+    return bool(lib().svdq_set_gemm_pairs(1 if enable else 0))
 
 
 def quantize_act(x, smooth=None, L1t=None, gscale=None, *, out=None):

@@ -24,7 +24,7 @@ ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "-I", INCLUDE, "-I", CSRC,
          "--expt-relaxed-constexpr"]
 
-SOURCES = ["api.cu", "quantize.cu", "gemm.cu", "awq.cu"]
+SOURCES = ["api.cu", "quantize.cu", "gemm.cu", "gemm_pair.cu", "awq.cu"]
 
 
 def _newest(paths):

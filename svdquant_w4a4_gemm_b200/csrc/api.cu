@@ -46,6 +46,7 @@ DeviceInfo g_dev[kMaxDevices];
 std::mutex g_mu;
 uint64_t g_timeout_ns = 2000000000ull;
 int g_fault = 0;
+int g_gemm_pairs = 0;
 
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
                                    const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
@@ -140,6 +141,7 @@ svdq_status device_ctx(void* stream, LaunchCtx* ctx) {
   ctx->err_word = d.err_word;
   ctx->timeout_ns = g_timeout_ns;
   ctx->fault_flags = g_fault;
+  ctx->gemm_pairs = g_gemm_pairs;
   return SVDQ_OK;
 }
 
@@ -422,6 +424,13 @@ uint64_t svdq_set_wait_timeout_ns(uint64_t ns) {
   std::lock_guard<std::mutex> lk(g_mu);
   const uint64_t prev = g_timeout_ns;
   g_timeout_ns = ns ? ns : 2000000000ull;
+  return prev;
+}
+
+int svdq_set_gemm_pairs(int enable) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  const int prev = g_gemm_pairs;
+  g_gemm_pairs = enable ? 1 : 0;
   return prev;
 }
 

@@ -48,14 +48,13 @@
 //               clipped at the M and N edges) into the tile's output (one,
 //               or one of up to three parts: Q, K, V of a fused
 //               projection); then release the accumulator.
-#include "internal.h"
-#include "ptx.cuh"
+#include "gemm_common.cuh"
 
 namespace svdq {
 namespace {
 
 constexpr int kBM = 128;
-constexpr int kBKBytes = 128;  // 256 FP4 elements per FP4 step and row
+constexpr int kBKBytes = kGemmBKBytes;
 constexpr int kStages = 4;                 // ring slots
 constexpr int kProducers = 2;              // producer warps; slot s belongs to producer s % 2
 constexpr int kMmaWarp = kProducers;
@@ -65,34 +64,6 @@ constexpr int kEpiWarps = 4;
 constexpr int kThreads = 32 * (kProducers + 1 + kStagerWarps + kEpiWarps);
 constexpr uint32_t kATileBytes = kBM * kBKBytes;  // 16 KB
 constexpr int kMaxRegions = 8;
-
-struct GemmParams {
-  int M, N, K, r;
-  int tiles_n, tiles;     // output tiles along N, total
-  const uint8_t* sf_a;
-  const uint8_t* sf_w;
-  const float* gs_a;
-  const float* gs_w;
-  const uint16_t* bias;   // [N] or null
-  int n_part;             // split output: columns per part (tmap_y, tmap_y1, tmap_y2); 0 = one output
-  int fault;              // test hook: 1 = the first ring slot never fills
-  WaitCfg wait;
-};
-
-// GELU, tanh form, in fp32: 0.5·v·(1 + tanh(√(2/π)·(v + 0.044715·v³))).
-// The hardware tanh keeps the activation off the epilogue's critical path
-// (one MUFU op per element); its ~2^-11 relative error is below the bf16
-// rounding of the output that follows.
-__device__ __forceinline__ float gelu_tanh(float v) {
-  const float u = 0.7978845608028654f * fmaf(0.044715f * v, v * v, v);
-  const float h = 0.5f * v;
-  return fmaf(h, tanh_approx(u), h);
-}
-
-__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
-  __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
-  return *reinterpret_cast<uint32_t*>(&h);
-}
 
 template <int BN>
 struct Layout {
@@ -354,14 +325,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     int rg = 0;                              // scale region of the next FP4 step
     uint32_t free_par = 0;                   // parity of each region's next sffree phase
     bool ok = true;
-    // One FP4 step: the slot's scales into region rg.  Per 64-K block kk this
-    // lane needs line `lane` (16 bytes) of the activation block and the words
-    // of the weight blocks that hold tile rows 32j + lane: weight row n0 + 32j
-    // + lane sits in word ((n0 % 128 + 32j) % 128) / 32 of line `lane` of
-    // block (n0 + 32j) / 128.  BN = 128: the whole line of the one block.
-    // BN = 192, n0 % 128 == 0: the line of block 0 (rows 0-127), then words
-    // 0-1 of block 1 (rows 128-191); n0 % 128 == 64: words 2-3 of block 0
-    // (rows 0-63), then the line of block 1 (rows 64-191).
+    // One FP4 step: the slot's scales into region rg (stage_scales).
     auto fp4_step = [&](bool hi64, int s, uint32_t ph) -> bool {
       // region rg's previous user is FP4 step f - kRegions
       if (f >= L::kRegions) {
@@ -371,49 +335,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!mbar_wait(&full_sf[s], (sf_par >> s) & 1u, p.wait, kErrTimeoutFull)) return false;
       sf_par ^= 1u << s;
       tc_fence_after();
-      const uint8_t* sa = stage_sfa(s) + lane * 16;
-      const uint8_t* sb = stage_sfb(s) + lane * 16;
-      uint32_t va[16];
-#pragma unroll
-      for (int kk = 0; kk < 4; ++kk) {
-        const uint4 u = *reinterpret_cast<const uint4*>(sa + kk * 512);
-        va[4 * kk] = u.x;
-        va[4 * kk + 1] = u.y;
-        va[4 * kk + 2] = u.z;
-        va[4 * kk + 3] = u.w;
-      }
-      const uint32_t sfr = tmem + lane_off + L::kSfCol + rg * L::kSfRegionCols;
-      // SFA: column 4kk + j = bytes [4j, 4j + 4) of line `lane` of block kk
-      tmem_st_32x32b_x16(sfr, va);
-      // SFB: column 16 + (BN/32)kk + j holds tile row 32j + lane
-      if constexpr (BN == 128) {
-        uint32_t vb[16];
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {
-          const uint4 x = *reinterpret_cast<const uint4*>(sb + kk * 512);
-          vb[4 * kk] = x.x;
-          vb[4 * kk + 1] = x.y;
-          vb[4 * kk + 2] = x.z;
-          vb[4 * kk + 3] = x.w;
-        }
-        tmem_st_32x32b_x16(sfr + 16, vb);
-      } else {
-        uint32_t vb[24];
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {
-          const uint4 x = *reinterpret_cast<const uint4*>(sb + (hi64 ? 2048 : 0) + kk * 512);
-          const uint2 y = *reinterpret_cast<const uint2*>(sb + (hi64 ? 8 : 2048) + kk * 512);
-          const uint32_t lo[6] = {x.x, x.y, x.z, x.w, y.x, y.y};
-          const uint32_t hi[6] = {y.x, y.y, x.x, x.y, x.z, x.w};
-#pragma unroll
-          for (int j = 0; j < 6; ++j) vb[6 * kk + j] = hi64 ? hi[j] : lo[j];
-        }
-        const uint32_t v16[16] = {vb[0], vb[1], vb[2],  vb[3],  vb[4],  vb[5],  vb[6],  vb[7],
-                                  vb[8], vb[9], vb[10], vb[11], vb[12], vb[13], vb[14], vb[15]};
-        const uint32_t v8[8] = {vb[16], vb[17], vb[18], vb[19], vb[20], vb[21], vb[22], vb[23]};
-        tmem_st_32x32b_x16(sfr + 16, v16);
-        tmem_st_32x32b_x8(sfr + 32, v8);
-      }
+      stage_scales<BN>(stage_sfa(s), stage_sfb(s), lane, hi64, true,
+                       tmem + lane_off + L::kSfCol + rg * L::kSfRegionCols);
       tmem_st_wait();
       tc_fence_before();
       // the MMA thread waits on sfready alone: make it imply the operands too
@@ -443,35 +366,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             ok = false;
             break;
           }
-          // this row's 32 fp32 values sit unswizzled in its own 128 bytes:
-          // read them all, then overwrite the same bytes with hi | lo
-          uint8_t* arow = stage_a(s) + row * 128;
-          float w[32];
-#pragma unroll
-          for (int q = 0; q < 8; ++q) {
-            const float4 u = *reinterpret_cast<const float4*>(arow + 16 * q);
-            w[4 * q] = u.x;
-            w[4 * q + 1] = u.y;
-            w[4 * q + 2] = u.z;
-            w[4 * q + 3] = u.w;
-          }
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {  // chunk q: hi of columns 8q..8q+7; chunk 4+q: their lo
-            uint32_t hw[4], lw[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const float t0 = __fmul_rn(w[8 * q + 2 * e], gprod);
-              const float t1 = __fmul_rn(w[8 * q + 2 * e + 1], gprod);
-              const float h0 = __bfloat162float(__float2bfloat16_rn(t0));
-              const float h1 = __bfloat162float(__float2bfloat16_rn(t1));
-              hw[e] = pack_bf16x2(h0, h1);
-              lw[e] = pack_bf16x2(__fsub_rn(t0, h0), __fsub_rn(t1, h1));
-            }
-            *reinterpret_cast<uint4*>(arow + ((q ^ (row & 7)) << 4)) =
-                make_uint4(hw[0], hw[1], hw[2], hw[3]);
-            *reinterpret_cast<uint4*>(arow + (((4 + q) ^ (row & 7)) << 4)) =
-                make_uint4(lw[0], lw[1], lw[2], lw[3]);
-          }
+          lowrank_operand_row(stage_a(s) + row * 128, row, gprod);
           fence_proxy_async_smem();
           __syncwarp();
           if (lane == 0) mbar_arrive(&lrf[s]);
@@ -492,14 +387,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       int m0, n0;
       tile_coords(t, p.tiles_n, BN, m0, n0);
       const int a = local & 1;
-      // the output this tile goes to (a tile never straddles two parts)
-      const CUtensorMap* ymap = &tmap_y;
-      int ycol = n0;
-      if (p.n_part) {
-        const int part = n0 / p.n_part;
-        ycol = n0 - part * p.n_part;
-        ymap = part == 0 ? &tmap_y : (part == 1 ? &tmap_y1 : &tmap_y2);
-      }
+      int ycol;
+      const CUtensorMap* ymap = output_map(p, n0, &tmap_y, &tmap_y1, &tmap_y2, ycol);
       // the tile's bias columns into this warp's shared-memory copy
       for (int c = lane; c < BN; c += 32) {
         const int col = n0 + c;
@@ -513,32 +402,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int j = 0; j < L::kBoxes; ++j) {
         // α·acc + bias -> bf16 for columns [64j, 64j + 64) of this quadrant's rows
         uint32_t packed[32];
-#pragma unroll
-        for (int c = 0; c < 4; c += 2) {  // 16-column chunks, two per load pair
-          uint32_t v0[16], v1[16];
-          tmem_ld_32x32b_x16(taddr + 64 * j + c * 16, v0);
-          tmem_ld_32x32b_x16(taddr + 64 * j + (c + 1) * 16, v1);
-          tmem_ld_wait();
-#pragma unroll
-          for (int u = 0; u < 2; ++u) {
-            const uint32_t* av = u ? v1 : v0;
-            const uint4* b4 = reinterpret_cast<const uint4*>(bsl + 64 * j + (c + u) * 16);
-            const uint4 bb0 = b4[0], bb1 = b4[1];
-            const uint32_t bw[8] = {bb0.x, bb0.y, bb0.z, bb0.w, bb1.x, bb1.y, bb1.z, bb1.w};
-#pragma unroll
-            for (int e = 0; e < 8; ++e) {
-              float lo = __fadd_rn(__fmul_rn(__uint_as_float(av[2 * e]), alpha),
-                                   __uint_as_float(bw[e] << 16));
-              float hi = __fadd_rn(__fmul_rn(__uint_as_float(av[2 * e + 1]), alpha),
-                                   __uint_as_float(bw[e] & 0xFFFF0000u));
-              if (gelu) {
-                lo = gelu_tanh(lo);
-                hi = gelu_tanh(hi);
-              }
-              packed[(c + u) * 8 + e] = pack_bf16x2(lo, hi);
-            }
-          }
-        }
+        epilogue_box<gelu>(taddr + 64 * j, bsl + 64 * j, alpha, packed);
         if (j == L::kBoxes - 1) {  // the accumulator is drained: the MMAs may refill it
           tc_fence_before();
           __syncwarp();
@@ -547,10 +411,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // 32 x 64 staging box, 128-byte swizzle
         if (lane == 0) bulk_wait_group_read<0>();  // the previous store has read the box
         __syncwarp();
-#pragma unroll
-        for (int q = 0; q < 8; ++q)
-          *reinterpret_cast<uint4*>(brow + ((q ^ (lane & 7)) << 4)) =
-              make_uint4(packed[4 * q], packed[4 * q + 1], packed[4 * q + 2], packed[4 * q + 3]);
+        write_box(brow, lane, packed);
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) {
@@ -596,15 +457,21 @@ svdq_status launch_w4a4_gemm(const LaunchCtx& ctx, const uint8_t* q_act, const u
   // the tile width must divide every part (parts > 1: N/parts is a multiple of 128)
   const int64_t n_part = N / parts;
   const int bn = (n_part % 192 == 0) ? 192 : 128;
+  // 256-row tiles on SM pairs (when enabled) where the shape has at least
+  // two row blocks: 256 x 192 where 192 divides the part, else 256 x 128
+  const int pair_bn = n_part % 192 == 0 ? 192 : 128;
+  const bool pair = ctx.gemm_pairs && M > kBM && n_part % pair_bn == 0;
   CUtensorMap ta{}, tb{}, tl{}, ty{}, tr{}, ty1{}, ty2{};
   if (!make_tmap_2d(&ta, q_act, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, M, K / 2, K / 2, kBM, kBKBytes,
                     128))
     return SVDQ_ERR_CUDA;
-  if (!make_tmap_2d(&tb, q_w, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, N, K / 2, K / 2, bn, kBKBytes, 128))
+  // B (and L2ᵀ) boxes: the tile's rows, or on SM pairs the half each CTA loads
+  const uint32_t b_rows = static_cast<uint32_t>(pair ? pair_bn / 2 : bn);
+  if (!make_tmap_2d(&tb, q_w, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, N, K / 2, K / 2, b_rows, kBKBytes, 128))
     return SVDQ_ERR_CUDA;
   if (r > 0) {
     if (!make_tmap_2d(&tl, L2t, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, N, r,
-                      static_cast<uint64_t>(r) * 2, bn, 64, 128))
+                      static_cast<uint64_t>(r) * 2, b_rows, 64, 128))
       return SVDQ_ERR_CUDA;
   } else {
     tl = ta;
@@ -636,6 +503,7 @@ svdq_status launch_w4a4_gemm(const LaunchCtx& ctx, const uint8_t* q_act, const u
   p.n_part = parts > 1 ? static_cast<int>(n_part) : 0;
   p.fault = ctx.fault_flags;
   p.wait = WaitCfg{ctx.timeout_ns, ctx.err_word};
+  if (pair) return launch_w4a4_gemm_pair(ctx, ta, tb, tl, ty, tr, ty1, ty2, p, pair_bn, activation);
   if (activation == SVDQ_ACT_GELU_TANH)
     return bn == 192 ? launch_bn<192, SVDQ_ACT_GELU_TANH>(ctx, ta, tb, tl, ty, tr, ty1, ty2, p)
                      : launch_bn<128, SVDQ_ACT_GELU_TANH>(ctx, ta, tb, tl, ty, tr, ty1, ty2, p);

@@ -18,6 +18,7 @@ struct LaunchCtx {
   uint32_t* err_word;    // device error word of `device`
   uint64_t timeout_ns;   // bound on every in-kernel wait
   int fault_flags;       // test-only fault injection
+  int gemm_pairs;        // 1: W4A4 GEMM on SM pairs where the shape allows (svdq_set_gemm_pairs)
 };
 
 // Encode a 2-D tiled tensor map (row-major [rows, cols] of `elem_bytes`
