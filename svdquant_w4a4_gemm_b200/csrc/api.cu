@@ -213,6 +213,24 @@ bool make_tmap_2d(CUtensorMap* map, const void* base, CUtensorMapDataType dtype,
   return true;
 }
 
+bool make_tmap_3d_u8(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1, uint64_t d2,
+                     uint64_t s1, uint64_t s2, uint32_t b0, uint32_t b1, uint32_t b2, bool swizzle128) {
+  const cuuint64_t dims[3] = {d0, d1, d2};
+  const cuuint64_t strides[2] = {s1, s2};
+  const cuuint32_t box[3] = {b0, b1, b2};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  const CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides,
+                              box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                              swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    fail(SVDQ_ERR_CUDA, "cuTensorMapEncodeTiled (3-D) failed (%d) dims=%llu,%llu,%llu", (int)r,
+         (unsigned long long)d0, (unsigned long long)d1, (unsigned long long)d2);
+    return false;
+  }
+  return true;
+}
+
 }  // namespace svdq
 
 using namespace svdq;

@@ -28,6 +28,12 @@ bool make_tmap_2d(CUtensorMap* map, const void* base, CUtensorMapDataType dtype,
                   uint32_t elem_bytes, uint64_t rows, uint64_t cols, uint64_t row_stride_bytes,
                   uint32_t box_rows, uint32_t box_cols, int swizzle_bytes);
 
+// A 3-D tiled tensor map over bytes: dims (d0, d1, d2) with byte strides s1
+// (between d1 indices) and s2 (between d2 indices), box (b0, b1, b2), 128-byte
+// swizzle when swizzle128.  Returns false and sets the detail on error.
+bool make_tmap_3d_u8(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1, uint64_t d2,
+                     uint64_t s1, uint64_t s2, uint32_t b0, uint32_t b1, uint32_t b2, bool swizzle128);
+
 // Thread-local error detail (api.cu).
 svdq_status fail(svdq_status st, const char* fmt, ...);
 svdq_status check_launch(const char* what);

@@ -142,6 +142,47 @@ __device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t threads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
 }
 
+// Named barrier that also returns the AND of `pred` over its threads.
+__device__ __forceinline__ bool named_bar_and(uint32_t id, uint32_t threads, bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "barrier.red.and.pred q, %2, %3, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"(static_cast<uint32_t>(pred)), "r"(id), "r"(threads)
+      : "memory");
+  return r != 0;
+}
+
+// Two IEEE single-precision products, each rounded to nearest even (the
+// same results as two __fmul_rn), in one packed instruction.
+__device__ __forceinline__ void mul_rn_x2(float a0, float a1, float b0, float b1, float& c0, float& c1) {
+  uint64_t r;
+  asm("{\n\t.reg .b64 x, y;\n\t"
+      "mov.b64 x, {%1, %2};\n\t"
+      "mov.b64 y, {%3, %4};\n\t"
+      "mul.rn.f32x2 %0, x, y;\n\t}"
+      : "=l"(r)
+      : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+  c0 = __uint_as_float(static_cast<uint32_t>(r));
+  c1 = __uint_as_float(static_cast<uint32_t>(r >> 32));
+}
+
+// RN(a / 6) for finite a >= 0, by one Markstein correction step (P. W.
+// Markstein, "Computation of elementary functions on the IBM RISC System/6000
+// processor", IBM J. Res. Dev. 34(1), 1990): q0 = RN(a·y) with y = RN(1/6),
+// the residual r = a − 6·q0 is exact in one FMA, and q0 + r·y rounded once is
+// RN(a/6) whenever a/6 is a normal number.  Below that the IEEE division.
+__device__ __forceinline__ float div6_rn(float a) {
+  if (a < 0x1.8p-124f) return __fdiv_rn(a, 6.0f);  // a/6 below 2^-126
+  const float y = 0x1.555556p-3f;                  // RN(1/6)
+  const float q0 = __fmul_rn(a, y);
+  const float r = __fmaf_rn(-q0, 6.0f, a);
+  return __fmaf_rn(r, y, q0);
+}
+
 // One thread per CTA: arrive at a grid-wide barrier (a counter that is zero
 // at launch) and wait, bounded, until `expected` CTAs have arrived.  Only for
 // kernels whose CTAs are all resident at once (cooperative launch).
@@ -177,6 +218,15 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* m, uin
       "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
       " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(dst)),
       "l"(reinterpret_cast<uint64_t>(m)), "r"(smem_u32(bar)), "r"(c0), "r"(c1)
+      : "memory");
+}
+
+__device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* m, uint64_t* bar, int32_t c0,
+                                            int32_t c1, int32_t c2) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(m)), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2)
       : "memory");
 }
 

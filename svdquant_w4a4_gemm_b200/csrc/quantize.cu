@@ -23,18 +23,20 @@
 //                the quantized tile's bf16(x̂) and the L1ᵀ slice into a TMEM
 //                accumulator; a new accumulator (of two) per run of
 //                sub-tiles in the same 128-row block ("segment").
-//   warps 2-9    quantizers, one sub-tile per warp (so up to 8 sub-tiles are
-//                worked on at once; with all warps on one sub-tile, each
-//                sub-tile costs a full dependent chain of latencies).  As many
-//                of them work as the ring has slots (at most 8), sub-tile i
-//                going to warp i mod slots: a warp then owns its ring slot,
-//                and the previous phase of every barrier it waits on is one
-//                it consumed itself (a parity wait cannot tell a phase from
-//                the one two before it, so a warp must never wait on a slot
-//                whose previous load may still be outstanding).  Lane l
-//                takes rows l, l+32, l+64, l+96 and each row's four 16-element
-//                groups: x̂ = x·inv_s, group max, E4M3 scale
-//                (cvt.rn.satfinite.e4m3x2; RN(gs / scale) from a per-CTA
+//   warps 2-9    quantizers, two warps per sub-tile (64 rows each), so up
+//                to ns/2 sub-tiles are worked on at once and a CTA's 10-11
+//                sub-tiles split into ~21 half-tiles: the last round is half
+//                as long.  Warp pair pq takes ring items pq, pq + ns/2, ...
+//                in slots i mod ns: a pair owns two slots, and the previous
+//                phase of every barrier it waits on is one it consumed itself
+//                (a parity wait cannot tell a phase from the one two before
+//                it, so a warp must never wait on a slot whose previous load
+//                may still be outstanding).  The pair agrees on each wait's
+//                verdict and meets before one of its warps releases the slot.
+//                Lane l takes rows 64h + l and 64h + l + 32 and each row's
+//                four 16-element groups: x̂ = x·inv_s (packed f32x2 products),
+//                group max, E4M3 scale (RN(amax/6) by one Markstein correction
+//                step, cvt.rn.satfinite.e4m3x2; RN(gs / scale) from a per-CTA
 //                table of the 127 scale codes), E2M1 codes (cvt.rn.satfinite
 //                .e2m1x2), the row's 32 code bytes and 4 scale bytes (one
 //                word in the 128x4 block layout), and bf16(x̂) written back
@@ -54,7 +56,7 @@
 // phase B quantizes as above with the tensor-wide gs_a, reading x again,
 // now from L2 (the CTA's phase-B loads go out while it waits at the
 // barrier).  The ring runs through both phases as one sequence of 2n
-// items, item i in slot i mod ns, owned by quantizer warp i mod ns.
+// items, item i in slot i mod ns, taken by quantizer warp pair i mod ns/2.
 #include <cstdio>
 #include <mutex>
 
@@ -66,8 +68,8 @@ namespace {
 
 constexpr int kBM = 128;
 constexpr int kSubK = 64;
-constexpr int kQuantWarps = 8;   // one sub-tile each, so up to 8 in flight
-constexpr int kMaxStages = kQuantWarps;  // ring depth <= quantizer warps: one slot per warp
+constexpr int kQuantWarps = 8;   // two per sub-tile, so up to 4 in flight
+constexpr int kMaxStages = kQuantWarps;  // ring depth <= quantizer warps: two slots per warp pair
 constexpr int kEpiWarps = 4;
 constexpr int kThreads = 32 * (2 + kQuantWarps + kEpiWarps);
 constexpr uint32_t kXTileBytes = kBM * kSubK * 2;
@@ -267,31 +269,38 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp < 2 + kQuantWarps) {
     // ------------------------------------------------------ quantizers ----
     const int qw = warp - 2;
-    // Warp qw < ns quantizes whole sub-tiles (units i = qw, qw + ns, ...),
-    // all of them in ring slot qw, so up to ns sub-tiles are in flight at
-    // once and each lane has 16 independent groups to interleave: lane l
-    // takes rows l, l + 32, l + 64, l + 96 of the tile, each row's four
-    // 16-element groups.
+    // Two warps per sub-tile: pair pq = qw / 2 takes ring items i = pq, pq + P,
+    // pq + 2P, ... (P = ns / 2 pairs), item i in slot i % ns, so a pair owns
+    // slots pq and pq + P and every barrier phase it waits on follows one it
+    // consumed itself (a parity wait cannot tell a phase from the one two
+    // before it).  Warp half h = qw % 2 takes rows 64h .. 64h + 63 of the
+    // tile: lane l rows 64h + l and 64h + l + 32, each row's four 16-element
+    // groups.  The pair agrees on every wait's verdict and meets before one
+    // of its warps releases the slot.
     const size_t kbytes = static_cast<size_t>(p.K) / 2;
-    const int s = qw;
-    uint32_t ph = 0;
-    int i = qw;              // ring item
+    const int npairs = ns / 2;
+    const int pq = qw >> 1, hh = qw & 1;
+    const bool active = pq < npairs;
+    const uint32_t pair_bar = 2 + static_cast<uint32_t>(pq);  // named barrier of the pair (ids 2..5)
+    int i = pq;              // ring item
     float gsq = gs;
     if constexpr (kSinglePass) {
-      // phase A: max|x·inv_s| over this warp's sub-tiles; each slot is
-      // released as soon as it is read
+      // phase A: max|x·inv_s| over this warp's half sub-tiles; each slot is
+      // released as soon as both halves are read
       bool ok = true;
       float m8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-      for (; qw < ns && i < phase_b0; i += ns, ph ^= 1u) {
-        // one verdict per warp: lanes that disagree at the time limit must not split up
-        if (!__all_sync(0xffffffffu, mbar_wait(&full[s], ph, p.wait, kErrTimeoutFull))) {
+      for (; active && i < phase_b0; i += npairs) {
+        const int s = i % ns;
+        // one verdict per pair: warps that disagree at the time limit must not split up
+        const bool w_ok = __all_sync(0xffffffffu, mbar_wait(&full[s], (i / ns) & 1, p.wait, kErrTimeoutFull));
+        if (!named_bar_and(pair_bar, 64, w_ok)) {
           ok = false;
           break;
         }
         const float* isk = inv_s + ((u0 + i) % kblocks) * kSubK;
-#pragma unroll 2
-        for (int j = 0; j < 4; ++j) {
-          const int row = lane + 32 * j;
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+          const int row = 64 * hh + lane + 32 * j;
           const uint8_t* trow = xs + s * kXTileBytes + row * 128;
 #pragma unroll
           for (int g = 0; g < 4; ++g) {
@@ -302,15 +311,16 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
               const float4 iv = is4[q];
-              m8[2 * q] = fmaxf(m8[2 * q], fabsf(__fmul_rn(bf16lo(w[2 * q]), iv.x)));
-              m8[2 * q] = fmaxf(m8[2 * q], fabsf(__fmul_rn(bf16hi(w[2 * q]), iv.y)));
-              m8[2 * q + 1] = fmaxf(m8[2 * q + 1], fabsf(__fmul_rn(bf16lo(w[2 * q + 1]), iv.z)));
-              m8[2 * q + 1] = fmaxf(m8[2 * q + 1], fabsf(__fmul_rn(bf16hi(w[2 * q + 1]), iv.w)));
+              float a0, a1, a2, a3;
+              mul_rn_x2(bf16lo(w[2 * q]), bf16hi(w[2 * q]), iv.x, iv.y, a0, a1);
+              mul_rn_x2(bf16lo(w[2 * q + 1]), bf16hi(w[2 * q + 1]), iv.z, iv.w, a2, a3);
+              m8[2 * q] = fmaxf(m8[2 * q], fmaxf(fabsf(a0), fabsf(a1)));
+              m8[2 * q + 1] = fmaxf(m8[2 * q + 1], fmaxf(fabsf(a2), fabsf(a3)));
             }
           }
         }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&empty[s]);
+        named_bar_sync(pair_bar, 64);
+        if (hh == 0 && lane == 0) mbar_arrive(&empty[s]);
       }
       float am = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
                        fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
@@ -344,15 +354,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else {
       if (p.gs_copy && blockIdx.x == 0 && threadIdx.x == 64) *p.gs_copy = gs;
     }
-    for (; qw < ns && i < n_items; i += ns, ph ^= 1u) {
+    for (; active && i < n_items; i += npairs) {
+      const int s = i % ns;
       const int u = u0 + i - phase_b0;
-      if (!__all_sync(0xffffffffu, mbar_wait(&full[s], ph, p.wait, kErrTimeoutFull))) break;
+      const bool w_ok = __all_sync(0xffffffffu, mbar_wait(&full[s], (i / ns) & 1, p.wait, kErrTimeoutFull));
+      if (!named_bar_and(pair_bar, 64, w_ok)) break;
       const int rb = u / kblocks, kb = u % kblocks;
       const float* isk = inv_s + kb * kSubK;
       uint8_t* sfb = p.sf_out + (static_cast<size_t>(rb) * kblocks + kb) * 512 + lane * 16;
-#pragma unroll 2
-      for (int j = 0; j < 4; ++j) {
-        const int row = lane + 32 * j;
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        const int row = 64 * hh + lane + 32 * j;
         const int grow = rb * kBM + row;
         uint8_t* trow = xs + s * kXTileBytes + row * 128;
         uint32_t codes[8];
@@ -367,12 +379,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           float xh[16];
           const float4* is4 = reinterpret_cast<const float4*>(isk + 16 * g);
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
+          for (int q = 0; q < 4; ++q) {  // x̂ = x·inv_s, two IEEE products per instruction
             const float4 iv = is4[q];
-            xh[4 * q + 0] = __fmul_rn(bf16lo(w[2 * q]), iv.x);
-            xh[4 * q + 1] = __fmul_rn(bf16hi(w[2 * q]), iv.y);
-            xh[4 * q + 2] = __fmul_rn(bf16lo(w[2 * q + 1]), iv.z);
-            xh[4 * q + 3] = __fmul_rn(bf16hi(w[2 * q + 1]), iv.w);
+            mul_rn_x2(bf16lo(w[2 * q]), bf16hi(w[2 * q]), iv.x, iv.y, xh[4 * q], xh[4 * q + 1]);
+            mul_rn_x2(bf16lo(w[2 * q + 1]), bf16hi(w[2 * q + 1]), iv.z, iv.w, xh[4 * q + 2], xh[4 * q + 3]);
           }
           // group max as a tree (max is exact, so the order does not matter)
           float m8[8];
@@ -381,7 +391,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int e = 0; e < 4; ++e) m8[e] = fmaxf(m8[e], m8[e + 4]);
           const float amax = fmaxf(fmaxf(m8[0], m8[2]), fmaxf(m8[1], m8[3]));
-          const float t = __fmul_rn(__fdiv_rn(amax, 6.0f), gsq);
+          const float t = __fmul_rn(div6_rn(amax), gsq);
           const uint32_t sf = cvt_e4m3(t);
           const float inv = gs_over_d[sf & 127u];  // RN(gs / dec(sf)); 0 for a zero scale
           sfw |= sf << (8 * g);
@@ -392,7 +402,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int h = 0; h < 2; ++h) {
             float q8[8];
 #pragma unroll
-            for (int e = 0; e < 8; ++e) q8[e] = __fmul_rn(xh[8 * h + e], inv);
+            for (int e = 0; e < 8; e += 2) mul_rn_x2(xh[8 * h + e], xh[8 * h + e + 1], inv, inv, q8[e], q8[e + 1]);
             codes[2 * g + h] = cvt_e2m1x8(q8);
           }
           if (has_lr) {  // bf16(x̂) back over the tile, for the down-projection
@@ -410,16 +420,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         // the row's four scales: bytes (row % 32)·16 + (row / 32)·4 + g of the
         // 512-byte block; rows past M inside the last 128-row block hold
         // zero-filled x, so their scales are the zero padding the layout needs
-        *reinterpret_cast<uint32_t*>(sfb + 4 * j) = sfw;
+        *reinterpret_cast<uint32_t*>(sfb + 4 * (2 * hh + j)) = sfw;
       }
-      if (has_lr) {
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&qdone[s]);
-      } else {
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&empty[s]);
-      }
+      if (has_lr) fence_proxy_async_smem();
+      named_bar_sync(pair_bar, 64);  // both halves done
+      if (hh == 0 && lane == 0) mbar_arrive(has_lr ? &qdone[s] : &empty[s]);
     }
   } else {
     // ------------------------------------------------- xl epilogue ----
@@ -512,7 +517,7 @@ int quantize_stages(int64_t K, int r) {
   const size_t fixed = quantize_fixed_bytes(K);
   const size_t per = kXTileBytes + static_cast<size_t>(r) * 128;
   const int fit = fixed < kSmemLimit ? static_cast<int>((kSmemLimit - fixed) / per) : 0;
-  return std::max(2, std::min(kMaxStages, fit));
+  return std::max(2, std::min(kMaxStages, fit)) & ~1;  // even: a warp pair owns two slots
 }
 }  // namespace
 

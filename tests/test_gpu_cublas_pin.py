@@ -85,12 +85,12 @@ def test_oracle_bytes_read_by_cublaslt_give_the_oracle_product(case):
 def test_library_gemm_matches_cublaslt_on_the_quantize_kernels_bytes(case):
     """The quantize kernel's codes and scales with the oracle's weight bytes:
     the library's W4A4 GEMM at r = 0 without bias equals cuBLASLt's result
-    times α = 1/(gs_a·gs_w).  Both sum the same exact products in fp32, so
-    they differ by the output roundings: the library's bf16(α·acc) is within
-    2^-9·|y| of α·acc, and a bf16 cuBLASLt output adds another 2^-9·|y|
-    before α is applied; the accumulation order adds ~1e-6 relative.  Each
-    element is held to that bound (plus 1e-4·rms for the order), and the
-    whole to the relative Frobenius bar."""
+    times α = 1/(gs_a·gs_w) within the output bar.  Both are tensor-core sums
+    of the same products, but with their own K order and internal
+    accumulation (measured: up to ~7e-3·rms apart element-wise, far above
+    two bf16 roundings), so the elements are held to the GEMM bar, not to a
+    rounding bound; a wrong layout or nibble order gives errors of order the
+    output's rms and fails it."""
     d = workloads.draw_svdq(case)
     L = prep.prepare_svdq_layer(d["x_cal"], d["W"], None, 0)
     w = weights_from_layer(L)
@@ -101,13 +101,6 @@ def test_library_gemm_matches_cublaslt_on_the_quantize_kernels_bytes(case):
     y_cb, which = cublas_nvfp4(qa, sfa, w.q_w, w.sf_w, M, N, K)
     alpha = 1.0 / (np.float64(gs_a) * np.float64(L["gs_w"]))
     ref = y_cb.double().cpu().numpy() * alpha
-    y = y_lib.double().cpu().numpy()
-    rounding = 2.0 ** -9 if y_cb.dtype == torch.float32 else 2.0 ** -8
-    rms = np.sqrt(np.mean(ref ** 2))
-    excess = np.abs(y - ref) - (rounding * np.abs(ref) + 1e-4 * rms)
-    assert excess.max() <= 0, f"library GEMM vs cuBLASLt ({which}): {int((excess > 0).sum())} elements " \
-                              f"beyond the rounding bound, worst by {excess.max() / rms:.3e}·rms"
-    rel_f = np.linalg.norm(y - ref) / np.linalg.norm(ref)
-    assert rel_f <= 5e-3, (which, rel_f)
+    assert_gemm_close(y_lib, ref, f"library GEMM vs cuBLASLt ({which})")
     torch.cuda.synchronize()
     sv.check_device_errors()
