@@ -309,6 +309,22 @@ uint64_t svdq_set_wait_timeout_ns(uint64_t ns);
 int svdq_set_gemm_pairs(int enable);
 
 /*
+ * svdq_set_pdl — whether later launches from this process allow
+ * programmatic dependent launch (CUDA's launch attribute
+ * programmaticStreamSerialization; default 1).  With it a kernel of this
+ * library may be scheduled onto the GPU while the kernel before it on the
+ * stream is still finishing; it initialises its barriers, allocates its
+ * tensor memory and prefetches its tensor-map descriptors, then waits for
+ * that kernel to complete and its writes to be visible (griddepcontrol.wait)
+ * before it touches any operand in global memory, so every argument keeps
+ * plain stream-order semantics.  Each kernel also signals at its start that
+ * the next one may be scheduled.  0 launches in plain stream order.  The
+ * pages have no counterpart (this is a launch property of the B200
+ * implementation).  Returns the previous setting.  Host-only; never fails.
+ */
+int svdq_set_pdl(int enable);
+
+/*
  * svdq_debug_set_fault — TEST HOOK.  flags = 1 makes the next launches of
  * svdq_w4a4_linear skip one producer arrive so that the consumer's bounded
  * wait runs out; flags = 2 makes the first CTA of the next

@@ -48,6 +48,7 @@ _SIGNATURES = {
     "svdq_check_device_errors": (_int, [_vp]),
     "svdq_set_wait_timeout_ns": (_u64, [_u64]),
     "svdq_set_gemm_pairs": (_int, [_int]),
+    "svdq_set_pdl": (_int, [_int]),
     "svdq_debug_set_fault": (_int, [_int]),
 }
 
@@ -105,6 +106,13 @@ def set_gemm_pairs(enable):
     (default off: one-SM tiles measured faster on B200); returns the previous
     setting."""
     return bool(lib().svdq_set_gemm_pairs(1 if enable else 0))
+
+
+def set_pdl(enable):
+    """Programmatic dependent launch for later launches (default on: a kernel
+    sets up while the previous one finishes, then waits for it before touching
+    any operand); returns the previous setting."""
+    return bool(lib().svdq_set_pdl(1 if enable else 0))
 
 
 def quantize_act(x, smooth=None, L1t=None, gscale=None, *, out=None):

@@ -47,6 +47,7 @@ std::mutex g_mu;
 uint64_t g_timeout_ns = 2000000000ull;
 int g_fault = 0;
 int g_gemm_pairs = 0;
+int g_pdl = 1;
 
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
                                    const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
@@ -142,6 +143,7 @@ svdq_status device_ctx(void* stream, LaunchCtx* ctx) {
   ctx->timeout_ns = g_timeout_ns;
   ctx->fault_flags = g_fault;
   ctx->gemm_pairs = g_gemm_pairs;
+  ctx->pdl = g_pdl;
   return SVDQ_OK;
 }
 
@@ -449,6 +451,13 @@ int svdq_set_gemm_pairs(int enable) {
   std::lock_guard<std::mutex> lk(g_mu);
   const int prev = g_gemm_pairs;
   g_gemm_pairs = enable ? 1 : 0;
+  return prev;
+}
+
+int svdq_set_pdl(int enable) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  const int prev = g_pdl;
+  g_pdl = enable ? 1 : 0;
   return prev;
 }
 

@@ -131,6 +131,8 @@ __global__ void __launch_bounds__(kThreads, 2)
                      const __half* __restrict__ scales, const __half* __restrict__ zeros,
                      const uint16_t* __restrict__ bias, int N, uint16_t* __restrict__ y) {
   extern __shared__ uint2 bfrag[];  // [K/64][4 steps][32 lanes][NT]; then the K-split partials
+  pdl_launch_dependents();
+  pdl_wait();  // global memory only after the previous kernel on the stream is done
   const int groups = K / 64;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int g = lane >> 2, t = lane & 3;
@@ -352,6 +354,7 @@ __global__ void __launch_bounds__(kSThreads, 1)
   const int s1 = static_cast<int>((static_cast<int64_t>(blockIdx.x + 1) * nstrips) / gridDim.x);
   const int nmine = s1 - s0;
 
+  pdl_launch_dependents();
   if (threadIdx.x == 0) {
     for (int s = 0; s < L.stages; ++s) {
       mbar_init(&full[s], 1);
@@ -365,6 +368,7 @@ __global__ void __launch_bounds__(kSThreads, 1)
     fence_mbar_init();
   }
   __syncthreads();
+  pdl_wait();  // global memory only after the previous kernel on the stream is done
 
   if (warp == kSProducer) {
     // ------------------------------------------------------ producer ----
@@ -609,11 +613,10 @@ svdq_status launch_stream(const LaunchCtx& ctx, const void* x, int M, int K, con
                        static_cast<uint64_t>(K) / 2, 128, 128, kSRows, static_cast<uint32_t>(L.chunks), true))
     return SVDQ_ERR_CUDA;
   const int grid = std::min(N / kSRows, ctx.num_sms);
-  kern<<<grid, kSThreads, smem, ctx.stream>>>(
-      tq, static_cast<const uint16_t*>(x), M, K, ainv, static_cast<const __half*>(scales),
-      static_cast<const __half*>(zeros), static_cast<const uint16_t*>(bias), N, static_cast<uint16_t*>(y),
-      WaitCfg{ctx.timeout_ns, ctx.err_word});
-  return check_launch("awq_w4a16_stream_kernel");
+  return launch_kernel(ctx, "awq_w4a16_stream_kernel", kern, dim3(grid), dim3(kSThreads), smem, tq,
+                       static_cast<const uint16_t*>(x), M, K, ainv, static_cast<const __half*>(scales),
+                       static_cast<const __half*>(zeros), static_cast<const uint16_t*>(bias), N,
+                       static_cast<uint16_t*>(y), WaitCfg{ctx.timeout_ns, ctx.err_word});
 }
 }  // namespace
 
@@ -650,11 +653,10 @@ svdq_status launch_awq_w4a16(const LaunchCtx& ctx, const void* x, int64_t M, int
                       static_cast<size_t>(kSplit - 1) * kTilesPerCta * 32 * 4 * nt * sizeof(float);
   auto kern = nt == 1 ? awq_w4a16_kernel<1> : awq_w4a16_kernel<2>;
   if (svdq_status e = set_smem_attr(ctx, reinterpret_cast<const void*>(kern), 227 * 1024)) return e;
-  kern<<<grid, kThreads, smem, ctx.stream>>>(
-      static_cast<const uint16_t*>(x), static_cast<int>(M), static_cast<int>(K), act_scale_inv,
-      qweight, static_cast<const __half*>(scales), static_cast<const __half*>(zeros),
-      static_cast<const uint16_t*>(bias), static_cast<int>(N), static_cast<uint16_t*>(y));
-  return check_launch("awq_w4a16_kernel");
+  return launch_kernel(ctx, "awq_w4a16_kernel", kern, dim3(grid), dim3(kThreads), smem,
+                       static_cast<const uint16_t*>(x), static_cast<int>(M), static_cast<int>(K), act_scale_inv,
+                       qweight, static_cast<const __half*>(scales), static_cast<const __half*>(zeros),
+                       static_cast<const uint16_t*>(bias), static_cast<int>(N), static_cast<uint16_t*>(y));
 }
 
 }  // namespace svdq

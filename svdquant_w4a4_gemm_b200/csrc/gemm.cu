@@ -131,6 +131,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int nk = (kblocks + 3) / 4;          // FP4 steps per tile (the last may be short)
   const int nsteps = nk + nlr;               // ring steps per tile
 
+  pdl_launch_dependents();
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&full[s], 1);
@@ -163,6 +164,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  pdl_wait();  // global memory only after the previous kernel on the stream is done
 
   if (warp < kProducers) {
     // ------------------------------------------------------ producers ----
@@ -443,8 +445,8 @@ svdq_status launch_bn(const LaunchCtx& ctx, const CUtensorMap& ta, const CUtenso
   p.tiles_n = (p.N + BN - 1) / BN;
   p.tiles = p.tiles_n * ((p.M + kBM - 1) / kBM);
   const int grid = std::min(p.tiles, ctx.num_sms);
-  w4a4_gemm_kernel<BN, ACT><<<grid, kThreads, smem, ctx.stream>>>(ta, tb, tl, ty, tr, ty1, ty2, p);
-  return check_launch("w4a4_gemm_kernel");
+  return launch_kernel(ctx, "w4a4_gemm_kernel", w4a4_gemm_kernel<BN, ACT>, dim3(grid), dim3(kThreads), smem, ta,
+                       tb, tl, ty, tr, ty1, ty2, p);
 }
 
 }  // namespace

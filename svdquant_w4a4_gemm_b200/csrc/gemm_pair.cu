@@ -127,6 +127,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   const int nk = (kblocks + 3) / 4;        // FP4 steps per tile (the last may be short)
   const int nsteps = nk + nlr;
 
+  pdl_launch_dependents();
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&full[s], 1);
@@ -161,6 +162,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   cluster_sync_all();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  pdl_wait();  // global memory only after the previous kernel on the stream is done
 
   if (warp < kProducers) {
     // ------------------------------------------------------ producers ----
@@ -466,9 +468,8 @@ svdq_status launch_act(const LaunchCtx& ctx, const CUtensorMap& ta, const CUtens
   p.tiles_n = p.N / BN;
   p.tiles = p.tiles_n * ((p.M + 2 * kBM - 1) / (2 * kBM));
   const int clusters = std::min(p.tiles, pair_clusters(ctx, fn, L::kSmemBytes));
-  w4a4_gemm_pair_kernel<BN, ACT><<<2 * clusters, kThreads, L::kSmemBytes, ctx.stream>>>(ta, tb, tl, ty, tr,
-                                                                                          ty1, ty2, p);
-  return check_launch("w4a4_gemm_pair_kernel");
+  return launch_kernel(ctx, "w4a4_gemm_pair_kernel", w4a4_gemm_pair_kernel<BN, ACT>, dim3(2 * clusters),
+                       dim3(kThreads), L::kSmemBytes, ta, tb, tl, ty, tr, ty1, ty2, p);
 }
 
 }  // namespace

@@ -1,6 +1,8 @@
 // internal.h — host-side plumbing shared by the library's translation units.
 #pragma once
 
+#include <utility>
+
 #include <cstdint>
 #include <cuda.h>
 #include <cuda_runtime.h>
@@ -19,6 +21,7 @@ struct LaunchCtx {
   uint64_t timeout_ns;   // bound on every in-kernel wait
   int fault_flags;       // test-only fault injection
   int gemm_pairs;        // 1: W4A4 GEMM on SM pairs where the shape allows (svdq_set_gemm_pairs)
+  int pdl;               // 1: launches may overlap the previous kernel's tail (svdq_set_pdl)
 };
 
 // Encode a 2-D tiled tensor map (row-major [rows, cols] of `elem_bytes`
@@ -37,6 +40,32 @@ bool make_tmap_3d_u8(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d
 // Thread-local error detail (api.cu).
 svdq_status fail(svdq_status st, const char* fmt, ...);
 svdq_status check_launch(const char* what);
+
+// Launches kern<<<grid, block, smem, ctx.stream>>>(args...) through
+// cudaLaunchKernelEx, with programmatic dependent launch allowed when
+// ctx.pdl: the kernel may then be scheduled while the previous kernel on the
+// stream is still finishing.  Every kernel of this library waits for its
+// predecessor (griddepcontrol.wait) before its first global memory access,
+// so stream order holds for every operand; what overlaps is the launch and
+// the set-up (barrier initialisation, tensor memory allocation, descriptor
+// prefetch).  A kernel compiled with __cluster_dims__ keeps its clusters.
+template <typename... KArgs, typename... Args>
+svdq_status launch_kernel(const LaunchCtx& ctx, const char* what, void (*kern)(KArgs...), dim3 grid,
+                          dim3 block, size_t smem, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = ctx.stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = ctx.pdl ? 1 : 0;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+  if (e != cudaSuccess) return fail(SVDQ_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+  return check_launch(what);
+}
 
 // Opt `kernel` in to `bytes` of dynamic shared memory in the current context
 // (once per context and kernel; thread-safe).  SVDQ_ERR_CUDA if refused.

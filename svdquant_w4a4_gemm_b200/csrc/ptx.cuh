@@ -93,6 +93,18 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const 
   }
 }
 
+// ------------------------------------------ programmatic dependent launch ----
+// Let the next kernel on the stream be scheduled (a no-op unless it was
+// launched with programmatic stream serialization).
+__device__ __forceinline__ void pdl_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// Wait until the previous kernel on the stream has completed and its memory
+// operations are visible (returns at once for a plain launch).  Every thread
+// that touches global memory passes here first.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // ------------------------------------------------------- CTA clusters ----
 // Rank of this CTA in its cluster.
 __device__ __forceinline__ uint32_t cluster_ctarank() {

@@ -147,6 +147,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   // Warp 0 sets up the barriers and issues the first ns loads right
   // away; the rest of the CTA fills the RN(1/s) and RN(gs/scale) tables in
   // the meantime.  Nobody else touches a barrier before the __syncthreads.
+  // Global memory only after the previous kernel on the stream is done.
+  pdl_launch_dependents();
   if (warp == 0 && lane == 0) {
     for (int s = 0; s < ns; ++s) {
       mbar_init(&full[s], 1);
@@ -160,6 +162,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     fence_mbar_init();
     tma_prefetch_desc(&tmap_x);
     if (has_lr) tma_prefetch_desc(&tmap_l1);
+    pdl_wait();
     for (int i = 0; i < min(n_items, ns); ++i) {
       const int u = u0 + (i < n_units ? i : i - n_units);
       const bool l1 = has_lr && i >= phase_b0;
@@ -169,6 +172,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (l1) tma_load_2d(ls + i * l1_bytes, &tmap_l1, &full[i], kb * kSubK, 0);
     }
   }
+  if (warp != 0 || lane != 0) pdl_wait();
   if (warp != 0) {
     // RN(1/s) for the columns of every sub-tile in [u0, u1): the whole K if
     // the range covers it, else per sub-tile (repeats write the same value)
@@ -472,6 +476,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 __global__ void __launch_bounds__(256) act_amax_kernel(const uint16_t* __restrict__ x, int M, int K,
                                                        int64_t ldx, const float* __restrict__ s,
                                                        unsigned* amax_bits) {
+  pdl_launch_dependents();
+  pdl_wait();
   const int c8 = blockIdx.x * blockDim.x + threadIdx.x;  // which 8-column chunk
   float m = 0.0f;
   if (c8 * 8 < K) {
@@ -501,6 +507,8 @@ __global__ void __launch_bounds__(256) act_amax_kernel(const uint16_t* __restric
 
 // Dynamic tensor scale, pass 3: turn the amax bits into gs in place.
 __global__ void act_scale_finalize_kernel(float* gs) {
+  pdl_launch_dependents();
+  pdl_wait();
   const float amax = __uint_as_float(*reinterpret_cast<unsigned*>(gs));
   *gs = tensor_scale_from_amax(amax);
 }
@@ -599,9 +607,10 @@ svdq_status launch_quantize_act(const LaunchCtx& ctx, const void* x, int64_t M, 
     if (cudaMemsetAsync(act_gscale_out, 0, 4, st) != cudaSuccess) return check_launch("memset gs");
     const int bx = static_cast<int>((K / 8 + 255) / 256);
     const int by = static_cast<int>(std::min<int64_t>(M, std::max(1, 4 * ctx.num_sms / bx)));
-    act_amax_kernel<<<dim3(bx, by), 256, 0, st>>>(static_cast<const uint16_t*>(x), p.M, p.K, ldx,
-                                                  smooth_s, reinterpret_cast<unsigned*>(act_gscale_out));
-    if (svdq_status e = check_launch("act_amax_kernel")) return e;
+    if (svdq_status e = launch_kernel(ctx, "act_amax_kernel", act_amax_kernel, dim3(bx, by), dim3(256), 0,
+                                      static_cast<const uint16_t*>(x), p.M, p.K, ldx, smooth_s,
+                                      reinterpret_cast<unsigned*>(act_gscale_out)))
+      return e;
   }
   const size_t smem = quantize_smem_bytes(K, r);
   {
@@ -638,11 +647,13 @@ svdq_status launch_quantize_act(const LaunchCtx& ctx, const void* x, int64_t M, 
     }
     return SVDQ_OK;
   }
-  quantize_act_kernel<false><<<grid, kThreads, smem, st>>>(tx, tl, p);
-  if (svdq_status e = check_launch("quantize_act_kernel")) return e;
+  if (svdq_status e = launch_kernel(ctx, "quantize_act_kernel", quantize_act_kernel<false>, dim3(grid),
+                                    dim3(kThreads), smem, tx, tl, p))
+    return e;
   if (!act_gscale) {
-    act_scale_finalize_kernel<<<1, 1, 0, st>>>(act_gscale_out);
-    if (svdq_status e = check_launch("act_scale_finalize_kernel")) return e;
+    if (svdq_status e = launch_kernel(ctx, "act_scale_finalize_kernel", act_scale_finalize_kernel, dim3(1),
+                                      dim3(1), 0, act_gscale_out))
+      return e;
   }
   return SVDQ_OK;
 }
