@@ -370,15 +370,24 @@ __global__ void __launch_bounds__(kSThreads, 1)
   __syncthreads();
   pdl_wait();  // global memory only after the previous kernel on the stream is done
 
+  // the consumers' loads of x go out before the weight stream: issued after
+  // it, they would wait behind it in the memory system and hold every
+  // consumer back by microseconds
+  constexpr uint32_t kXIssued = 1;                       // named barrier
+  constexpr uint32_t kXIssuedThreads = 32 * (kSWarps + 1);  // consumers + producer
   if (warp == kSProducer) {
     // ------------------------------------------------------ producer ----
-    // lane 0: 1/a, then the strips into the ring as slots come free
+    // lane 0: 1/a, then (once x is requested) the strips into the ring as
+    // slots come free
     if (lane == 0) {
       tma_prefetch_desc(&tmap_q);
       if (ainv) {
         mbar_arrive_expect_tx(abar, static_cast<uint32_t>(K * 4));
         bulk_load(ainv_s, ainv, static_cast<uint32_t>(K * 4), abar);
       }
+    }
+    named_bar_sync(kXIssued, kXIssuedThreads);
+    if (lane == 0) {
       const uint32_t bytes = static_cast<uint32_t>(L.qbytes + 2 * L.sbytes);
       int issued = 0;
       for (int i = 0; i < nmine; ++i) {
@@ -461,6 +470,7 @@ __global__ void __launch_bounds__(kSThreads, 1)
         xr[gi][s] = __ldg(reinterpret_cast<const uint4*>(x + off));
         if (!v) xr[gi][s] = make_uint4(0u, 0u, 0u, 0u);
       }
+    named_bar_arrive(kXIssued, kXIssuedThreads);
     if (ainv) __all_sync(0xffffffffu, mbar_wait(abar, 0, wait, kErrTimeoutFull));
 #pragma unroll
     for (int gi = 0; gi < GMAX; ++gi)

@@ -154,6 +154,12 @@ __device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t threads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
 }
 
+// Arrive at a named barrier without waiting (the threads that wait use
+// named_bar_sync with the same total count).
+__device__ __forceinline__ void named_bar_arrive(uint32_t id, uint32_t threads) {
+  asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
+
 // Named barrier that also returns the AND of `pred` over its threads.
 __device__ __forceinline__ bool named_bar_and(uint32_t id, uint32_t threads, bool pred) {
   uint32_t r;

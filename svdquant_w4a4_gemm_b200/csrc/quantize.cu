@@ -126,7 +126,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* ls = xs + ns * kXTileBytes;
   float* inv_s = reinterpret_cast<float*>(ls + ns * l1_bytes);        // [K], touched columns
   float* gs_over_d = inv_s + p.K;                                     // [128] by E4M3 code
-  uint64_t* full = reinterpret_cast<uint64_t*>(gs_over_d + 128);
+  uint8_t* cstage = reinterpret_cast<uint8_t*>(gs_over_d + 128);     // [kQuantWarps][32 rows][32 B]
+  uint64_t* full = reinterpret_cast<uint64_t*>(cstage + kQuantWarps * 1024);
   uint64_t* qdone = full + kMaxStages;
   uint64_t* empty = qdone + kMaxStages;
   uint64_t* acc_full = empty + kMaxStages;  // [2]
@@ -144,10 +145,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int phase_b0 = kSinglePass ? n_units : 0;   // first phase-B item
   const int n_items = phase_b0 + n_units;
 
-  // Warp 0 sets up the barriers and issues the first ns loads right
-  // away; the rest of the CTA fills the RN(1/s) and RN(gs/scale) tables in
-  // the meantime.  Nobody else touches a barrier before the __syncthreads.
-  // Global memory only after the previous kernel on the stream is done.
+  // Warp 0 sets up the barriers and issues the first ns loads as soon as
+  // the other warps have issued their own set-up loads (s and gs): issued
+  // after the x stream, those would wait behind it in the memory system and
+  // hold the tables, and so the quantizers, back by microseconds.  The rest
+  // of the CTA fills the RN(1/s) and RN(gs/scale) tables in the meantime.
+  // Nobody else touches an mbarrier before the __syncthreads.  Global memory
+  // only after the previous kernel on the stream is done.
+  constexpr uint32_t kSetupBar = 6;  // named barrier: the set-up loads are issued
   pdl_launch_dependents();
   if (warp == 0 && lane == 0) {
     for (int s = 0; s < ns; ++s) {
@@ -162,7 +167,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     fence_mbar_init();
     tma_prefetch_desc(&tmap_x);
     if (has_lr) tma_prefetch_desc(&tmap_l1);
-    pdl_wait();
+  }
+  pdl_wait();
+  const float gs_loaded = kSinglePass ? 1.0f : (p.gs_in ? *p.gs_in : tensor_scale_from_amax(*p.amax_src));
+  if (warp == 0) named_bar_sync(kSetupBar, kThreads);
+  if (warp == 0 && lane == 0) {
     for (int i = 0; i < min(n_items, ns); ++i) {
       const int u = u0 + (i < n_units ? i : i - n_units);
       const bool l1 = has_lr && i >= phase_b0;
@@ -172,18 +181,30 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (l1) tma_load_2d(ls + i * l1_bytes, &tmap_l1, &full[i], kb * kSubK, 0);
     }
   }
-  if (warp != 0 || lane != 0) pdl_wait();
   if (warp != 0) {
     // RN(1/s) for the columns of every sub-tile in [u0, u1): the whole K if
-    // the range covers it, else per sub-tile (repeats write the same value)
+    // the range covers it, else per sub-tile (repeats write the same value).
+    // Up to 8 columns a thread are loaded before the x stream goes out.
     const int t = threadIdx.x - 32, nt = kThreads - 32;
-    if (u1 - u0 >= kblocks) {
-      for (int j = t; j < p.K; j += nt) inv_s[j] = p.smooth_s ? __fdiv_rn(1.0f, p.smooth_s[j]) : 1.0f;
-    } else {
-      for (int j = t; j < (u1 - u0) * kSubK; j += nt) {
-        const int col = ((u0 + j / kSubK) % kblocks) * kSubK + j % kSubK;
-        inv_s[col] = p.smooth_s ? __fdiv_rn(1.0f, p.smooth_s[col]) : 1.0f;
-      }
+    const bool whole = u1 - u0 >= kblocks;
+    const int ncols = whole ? p.K : (u1 - u0) * kSubK;
+    auto column = [&](int j) { return whole ? j : ((u0 + j / kSubK) % kblocks) * kSubK + j % kSubK; };
+    constexpr int kEarly = 8;
+    float sv[kEarly];
+#pragma unroll
+    for (int e = 0; e < kEarly; ++e) {
+      const int j = t + e * nt;
+      sv[e] = (p.smooth_s && j < ncols) ? p.smooth_s[column(j)] : 1.0f;
+    }
+    named_bar_arrive(kSetupBar, kThreads);
+#pragma unroll
+    for (int e = 0; e < kEarly; ++e) {
+      const int j = t + e * nt;
+      if (j < ncols) inv_s[column(j)] = p.smooth_s ? __fdiv_rn(1.0f, sv[e]) : 1.0f;
+    }
+    for (int j = t + kEarly * nt; j < ncols; j += nt) {
+      const int col = column(j);
+      inv_s[col] = p.smooth_s ? __fdiv_rn(1.0f, p.smooth_s[col]) : 1.0f;
     }
   }
   if (warp == 1 && has_lr) {
@@ -200,7 +221,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     cta_amax_bits = 0u;
     grid_ok = 1;
   }
-  const float gs = kSinglePass ? 1.0f : (p.gs_in ? *p.gs_in : tensor_scale_from_amax(*p.amax_src));
+  const float gs = gs_loaded;
   if (threadIdx.x < 128 && !kSinglePass) {
     const float d = e4m3_to_f32(threadIdx.x);
     gs_over_d[threadIdx.x] = (d == 0.0f || threadIdx.x == 127) ? 0.0f : __fdiv_rn(gs, d);
@@ -366,6 +387,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int rb = u / kblocks, kb = u % kblocks;
       const float* isk = inv_s + kb * kSubK;
       uint8_t* sfb = p.sf_out + (static_cast<size_t>(rb) * kblocks + kb) * 512 + lane * 16;
+      uint8_t* stg = cstage + qw * 1024;  // this warp's 32 rows x 32 code bytes
 #pragma unroll
       for (int j = 0; j < 2; ++j) {
         const int row = 64 * hh + lane + 32 * j;
@@ -416,11 +438,22 @@ __global__ void __launch_bounds__(kThreads, 1)
                                                         pack_bf16x2(xh[12], xh[13]), pack_bf16x2(xh[14], xh[15]));
           }
         }
-        if (grow < p.M) {  // the row's 32 code bytes of this 64-column block
-          uint4* dst = reinterpret_cast<uint4*>(p.q_out + static_cast<size_t>(grow) * kbytes + kb * (kSubK / 2));
-          dst[0] = make_uint4(codes[0], codes[1], codes[2], codes[3]);
-          dst[1] = make_uint4(codes[4], codes[5], codes[6], codes[7]);
+        // the pass's 32 rows of 32 code bytes go out through shared memory,
+        // so that each store writes whole 32-byte rows (16 per instruction)
+        // instead of halves of 32 rows
+        reinterpret_cast<uint4*>(stg + lane * 32)[0] = make_uint4(codes[0], codes[1], codes[2], codes[3]);
+        reinterpret_cast<uint4*>(stg + lane * 32)[1] = make_uint4(codes[4], codes[5], codes[6], codes[7]);
+        __syncwarp();
+#pragma unroll
+        for (int k = 0; k < 2; ++k) {
+          const int rr = 16 * k + (lane >> 1);  // row of the pass; lane & 1: its half
+          const int g2 = rb * kBM + 64 * hh + 32 * j + rr;
+          const uint4 v = reinterpret_cast<const uint4*>(stg)[32 * k + lane];
+          if (g2 < p.M)
+            *reinterpret_cast<uint4*>(p.q_out + static_cast<size_t>(g2) * kbytes + kb * (kSubK / 2) +
+                                      (lane & 1) * 16) = v;
         }
+        __syncwarp();  // the next pass reuses the staging rows
         // the row's four scales: bytes (row % 32)·16 + (row / 32)·4 + g of the
         // 512-byte block; rows past M inside the last 128-row block hold
         // zero-filled x, so their scales are the zero padding the layout needs
@@ -506,6 +539,17 @@ __global__ void __launch_bounds__(256) act_amax_kernel(const uint16_t* __restric
 }
 
 // Dynamic tensor scale, pass 3: turn the amax bits into gs in place.
+// xl = 0 before the quantize kernel adds its partial sums (a row block's K
+// range spans several CTAs); a kernel rather than a memset node, so that
+// programmatic dependent launch chains it to its neighbours.
+__global__ void __launch_bounds__(256) zero_f32x4_kernel(float4* __restrict__ p, size_t n4) {
+  pdl_launch_dependents();
+  pdl_wait();
+  for (size_t i = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n4;
+       i += static_cast<size_t>(gridDim.x) * blockDim.x)
+    p[i] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+}
+
 __global__ void act_scale_finalize_kernel(float* gs) {
   pdl_launch_dependents();
   pdl_wait();
@@ -518,7 +562,7 @@ __global__ void act_scale_finalize_kernel(float* gs) {
 namespace {
 constexpr size_t kSmemLimit = 227 * 1024 - 64;  // less the kernel's static shared words
 size_t quantize_fixed_bytes(int64_t K) {
-  return 1024 + static_cast<size_t>(K) * 4 + 128 * 4 + 8 * (3 * kMaxStages + 4) + 16;
+  return 1024 + static_cast<size_t>(K) * 4 + 128 * 4 + kQuantWarps * 1024 + 8 * (3 * kMaxStages + 4) + 16;
 }
 // Ring depth: as many sub-tiles as fit next to the RN(1/s) table, 2..8.
 int quantize_stages(int64_t K, int r) {
@@ -598,8 +642,13 @@ svdq_status launch_quantize_act(const LaunchCtx& ctx, const void* x, int64_t M, 
   p.wait = WaitCfg{ctx.timeout_ns, ctx.err_word};
 
   cudaStream_t st = ctx.stream;
-  if (r > 0 && cudaMemsetAsync(lora_out, 0, static_cast<size_t>(M) * r * 4, st) != cudaSuccess)
-    return check_launch("memset lora_out");
+  if (r > 0) {  // lora_out is 16-byte aligned and M·r a multiple of 16
+    const size_t n4 = static_cast<size_t>(M) * r / 4;
+    const int blocks = static_cast<int>(std::min<size_t>((n4 + 255) / 256, 2 * static_cast<size_t>(ctx.num_sms)));
+    if (svdq_status e = launch_kernel(ctx, "zero_f32x4_kernel", zero_f32x4_kernel, dim3(blocks), dim3(256), 0,
+                                      reinterpret_cast<float4*>(lora_out), n4))
+      return e;
+  }
   if (single_pass) {
     if (cudaMemsetAsync(grid_sync, 0, 2 * sizeof(uint32_t), st) != cudaSuccess)
       return check_launch("memset workspace");
