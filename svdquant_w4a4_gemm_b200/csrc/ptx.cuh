@@ -205,16 +205,19 @@ __device__ __forceinline__ float div6_rn(float a) {
 // at launch) and wait, bounded, until `expected` CTAs have arrived.  Only for
 // kernels whose CTAs are all resident at once (cooperative launch).
 __device__ __forceinline__ bool grid_arrive_wait(uint32_t* ctr, uint32_t expected, const WaitCfg& w) {
-  __threadfence();  // this CTA's writes before its arrival
-  atomicAdd(ctr, 1u);
-  if (ld_acquire_gpu(ctr) >= expected) return true;
+  // one release add: this thread's earlier writes (the CTA's max) are visible
+  // to any thread that sees the count; the last arrival needs no poll
+  uint32_t old;
+  asm volatile("atom.add.release.gpu.global.u32 %0, [%1], 1;" : "=r"(old) : "l"(ctr) : "memory");
+  if (old + 1 >= expected) return true;
+  // the count comes back from L2 behind the phase-B loads already in flight,
+  // so poll without sleeping
   const uint64_t t0 = globaltimer();
   while (ld_acquire_gpu(ctr) < expected) {
     if (globaltimer() - t0 > w.timeout_ns) {
       atomicOr(w.err, kErrTimeoutGrid);
       return false;
     }
-    __nanosleep(64);
   }
   return true;
 }

@@ -391,7 +391,6 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
       for (int j = 0; j < 2; ++j) {
         const int row = 64 * hh + lane + 32 * j;
-        const int grow = rb * kBM + row;
         uint8_t* trow = xs + s * kXTileBytes + row * 128;
         uint32_t codes[8];
         uint32_t sfw = 0;  // the row's four scale bytes
@@ -540,11 +539,15 @@ __global__ void __launch_bounds__(256) act_amax_kernel(const uint16_t* __restric
 
 // Dynamic tensor scale, pass 3: turn the amax bits into gs in place.
 // xl = 0 before the quantize kernel adds its partial sums (a row block's K
-// range spans several CTAs); a kernel rather than a memset node, so that
-// programmatic dependent launch chains it to its neighbours.
-__global__ void __launch_bounds__(256) zero_f32x4_kernel(float4* __restrict__ p, size_t n4) {
+// range spans several CTAs), and the words the dynamic scale accumulates
+// into (the single-pass grid barrier's counter and max, or the max pass's
+// max); a kernel rather than memset nodes, so that programmatic dependent
+// launch chains it to its neighbours.
+__global__ void __launch_bounds__(256) clear_kernel(float4* __restrict__ p, size_t n4, uint32_t* __restrict__ words,
+                                                    int nwords) {
   pdl_launch_dependents();
   pdl_wait();
+  if (blockIdx.x == 0 && static_cast<int>(threadIdx.x) < nwords) words[threadIdx.x] = 0u;
   for (size_t i = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n4;
        i += static_cast<size_t>(gridDim.x) * blockDim.x)
     p[i] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
@@ -642,18 +645,19 @@ svdq_status launch_quantize_act(const LaunchCtx& ctx, const void* x, int64_t M, 
   p.wait = WaitCfg{ctx.timeout_ns, ctx.err_word};
 
   cudaStream_t st = ctx.stream;
-  if (r > 0) {  // lora_out is 16-byte aligned and M·r a multiple of 16
+  // lora_out is 16-byte aligned and M·r a multiple of 16; the dynamic scale's
+  // words: the workspace (single pass) or act_gscale_out (max pass)
+  uint32_t* words = single_pass ? grid_sync : (!act_gscale ? reinterpret_cast<uint32_t*>(act_gscale_out) : nullptr);
+  const int nwords = single_pass ? 2 : (!act_gscale ? 1 : 0);
+  if (r > 0 || nwords > 0) {
     const size_t n4 = static_cast<size_t>(M) * r / 4;
-    const int blocks = static_cast<int>(std::min<size_t>((n4 + 255) / 256, 2 * static_cast<size_t>(ctx.num_sms)));
-    if (svdq_status e = launch_kernel(ctx, "zero_f32x4_kernel", zero_f32x4_kernel, dim3(blocks), dim3(256), 0,
-                                      reinterpret_cast<float4*>(lora_out), n4))
+    const int blocks = static_cast<int>(
+        std::max<size_t>(1, std::min<size_t>((n4 + 255) / 256, 2 * static_cast<size_t>(ctx.num_sms))));
+    if (svdq_status e = launch_kernel(ctx, "clear_kernel", clear_kernel, dim3(blocks), dim3(256), 0,
+                                      reinterpret_cast<float4*>(lora_out), n4, words, nwords))
       return e;
   }
-  if (single_pass) {
-    if (cudaMemsetAsync(grid_sync, 0, 2 * sizeof(uint32_t), st) != cudaSuccess)
-      return check_launch("memset workspace");
-  } else if (!act_gscale) {
-    if (cudaMemsetAsync(act_gscale_out, 0, 4, st) != cudaSuccess) return check_launch("memset gs");
+  if (!single_pass && !act_gscale) {
     const int bx = static_cast<int>((K / 8 + 255) / 256);
     const int by = static_cast<int>(std::min<int64_t>(M, std::max(1, 4 * ctx.num_sms / bx)));
     if (svdq_status e = launch_kernel(ctx, "act_amax_kernel", act_amax_kernel, dim3(bx, by), dim3(256), 0,
