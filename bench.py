@@ -367,7 +367,7 @@ def bench_device(args, rank, world, dev):
 
         legs = None
         if world == 1 and not args.no_legs:
-            legs = bench_legs(sv, dev, l2, timer, sets)
+            legs = bench_legs(sv, dev, l2, timer, sets, args.only_legs)
         w2 = time.perf_counter()
     clocks = clk.summary()
     clocks["span"] = "whole measurement (timed steps, per-kernel timings, e2e, legs)"
@@ -388,8 +388,10 @@ def _tf(flops, t):
     return round(flops / t["us"] / 1e6, 1)
 
 
-def bench_legs(sv, dev, l2, timer, head_sets):
+def bench_legs(sv, dev, l2, timer, head_sets, only=None):
+    """The other workloads; `only`: a comma-separated subset of their names."""
     legs = {}
+    pick = set(only.split(",")) if only else None
     hbm = peaks().get("hbm_gbs", 6650.0)
     peak = fp4_peak(peaks())[0]
     for name, fn in (("tiny_layer", lambda: leg_tiny(sv, dev, l2, timer)),
@@ -399,6 +401,8 @@ def bench_legs(sv, dev, l2, timer, head_sets):
                      ("awq_w4a16", lambda: leg_awq(sv, dev, l2, timer, hbm)),
                      ("cublaslt_nvfp4", lambda: leg_cublaslt(sv, dev, timer, head_sets, peak)),
                      ("device_prep", lambda: leg_prep(dev))):
+        if pick is not None and name not in pick:
+            continue
         try:
             legs[name] = fn()
         except Exception as e:  # noqa: BLE001 - report it on the line, keep the line
@@ -734,6 +738,9 @@ def main():
     ap.add_argument("--no-legs", action="store_true", help="skip the other workloads")
     ap.add_argument("--legs", action="store_true", help=argparse.SUPPRESS)  # legs are the default
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--only-legs", default=None,
+                    help="comma-separated subset of the other workloads (tiny_layer, quantize_scale_variants, "
+                         "mlp, qkv_rank_sweep, awq_w4a16, cublaslt_nvfp4, device_prep)")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
     args.steps = max(1, args.steps)
@@ -801,7 +808,8 @@ def main():
         "timed_region_ms": round(res["total_ms"], 3),
         "e2e": {"value": res["e2e_tflops"], "unit": UNIT,
                 "h2d_bytes_per_step": res["h2d"], "d2h_bytes_per_step": res["d2h"]},
-        "gpu_launches": 2 * steps,
+        # per step: the xl clear kernel (r > 0), the quantize kernel, the GEMM
+        "gpu_launches": (3 if CASE.r > 0 else 2) * steps,
         "cpu_baseline": cpu,
     }
     if res["legs"]:
