@@ -242,17 +242,27 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t sf_par = 0;                   // parity of each region's next sfready phase
       uint32_t lr_par = 0;                   // parity of each slot's next lrf phase
       const int nkb_last = kblocks - 4 * (nk - 1);  // 64-K blocks of the last FP4 step
+      const int nk_full = nkb_last == 4 ? nk : nk - 1;  // FP4 steps of four MMAs
       const int lr_k = p.r < 32 ? 1 : 2;     // low-rank k-steps per slice (hi and lo each)
+      static_assert((kStages & (kStages - 1)) == 0, "the ring index wraps by a mask");
       auto advance = [&]() {
-        if (++s == kStages) {
-          s = 0;
-          soff = 0;
-        } else {
-          soff += L::kStage >> 4;
-        }
+        s = (s + 1) & (kStages - 1);
+        soff = static_cast<uint64_t>(s) * (L::kStage >> 4);
+      };
+      // the stagers arrive only after the slot's operands have landed
+      auto wait_scales = [&](bool ready) -> bool {
+        if (!ready && !mbar_wait(&sfready[rg], (sf_par >> rg) & 1u, p.wait, kErrTimeoutFull)) return false;
+        sf_par ^= 1u << rg;
+        tc_fence_after();
+        return true;
+      };
+      auto next_region = [&]() {
+        rg = rg + 1 == L::kRegions ? 0 : rg + 1;
+        sfr = tmem + L::kSfCol + static_cast<uint32_t>(rg) * L::kSfRegionCols;
       };
       int local = 0;                         // tiles done by this CTA
       bool ok = true;
+      bool ready = false;                    // the next FP4 step's sfready phase is known complete
       for (int t = blockIdx.x; ok && t < p.tiles; t += gridDim.x, ++local) {
         const int a = local & 1;
         const uint32_t acc = tmem + a * BN;
@@ -263,37 +273,43 @@ __global__ void __launch_bounds__(kThreads, 1)
           break;
         }
         tc_fence_after();
-        bool ready = false;                  // the next step's sfready phase is known complete
-        for (int st = 0; st < nk; ++st) {
-          // the stagers arrive only after the slot's operands have landed
-          if (!ready && !mbar_wait(&sfready[rg], (sf_par >> rg) & 1u, p.wait, kErrTimeoutFull)) {
+        // Full FP4 steps: straight-line code between the MMAs (a branch in
+        // the MMA stream costs tensor time even when it is not taken).  The
+        // next step's barrier is tested while the pipe is busy; a phase seen
+        // complete stays complete, across tiles too.
+        for (int st = 0; st < nk_full; ++st) {
+          if (!wait_scales(ready)) {
             ok = false;
             break;
           }
-          sf_par ^= 1u << rg;
-          tc_fence_after();
           const uint64_t da = da0 + soff, db = db0 + soff;
           const int rg_next = rg + 1 == L::kRegions ? 0 : rg + 1;
-          if (st + 1 < nk || nkb_last == 4) {
-            umma_nvfp4(acc, da, db, id_fp4, sfr, sfr + 16, st > 0 ? 1u : 0u);
-            umma_nvfp4(acc, da + 2, db + 2, id_fp4, sfr + 4, sfr + 16 + L::kSfbCols, 1u);
-            umma_nvfp4(acc, da + 4, db + 4, id_fp4, sfr + 8, sfr + 16 + 2 * L::kSfbCols, 1u);
-            // look at the next step's barrier while the tensor pipe is busy:
-            // waiting for it after the last MMA would leave the pipe idle
-            ready = st + 1 < nk && mbar_test(&sfready[rg_next], (sf_par >> rg_next) & 1u);
-            umma_nvfp4(acc, da + 6, db + 6, id_fp4, sfr + 12, sfr + 16 + 3 * L::kSfbCols, 1u);
-          } else {
-            ready = false;
-            for (int kk = 0; kk < nkb_last; ++kk)
-              umma_nvfp4(acc, da + 2 * kk, db + 2 * kk, id_fp4, sfr + 4 * kk,
-                         sfr + 16 + L::kSfbCols * kk, (st > 0 || kk > 0) ? 1u : 0u);
-          }
+          umma_nvfp4(acc, da, db, id_fp4, sfr, sfr + 16, st > 0 ? 1u : 0u);
+          umma_nvfp4(acc, da + 2, db + 2, id_fp4, sfr + 4, sfr + 16 + L::kSfbCols, 1u);
+          umma_nvfp4(acc, da + 4, db + 4, id_fp4, sfr + 8, sfr + 16 + 2 * L::kSfbCols, 1u);
+          ready = mbar_test(&sfready[rg_next], (sf_par >> rg_next) & 1u);
+          umma_nvfp4(acc, da + 6, db + 6, id_fp4, sfr + 12, sfr + 16 + 3 * L::kSfbCols, 1u);
           umma_commit(&empty[s]);
           umma_commit(&sffree[rg]);
-          rg = rg_next;
-          sfr = rg == 0 ? tmem + L::kSfCol : sfr + L::kSfRegionCols;
+          next_region();
           advance();
         }
+        if (ok && nk_full < nk) {  // the short last FP4 step (K % 256 != 0)
+          if (!wait_scales(ready)) {
+            ok = false;
+            break;
+          }
+          const uint64_t da = da0 + soff, db = db0 + soff;
+          for (int kk = 0; kk < nkb_last; ++kk)
+            umma_nvfp4(acc, da + 2 * kk, db + 2 * kk, id_fp4, sfr + 4 * kk, sfr + 16 + L::kSfbCols * kk,
+                       (nk_full > 0 || kk > 0) ? 1u : 0u);
+          umma_commit(&empty[s]);
+          umma_commit(&sffree[rg]);
+          ready = false;
+          next_region();
+          advance();
+        }
+        if (!ok) break;
         for (int j = 0; ok && j < nlr; ++j) {
           if (!mbar_wait(&lrf[s], (lr_par >> s) & 1u, p.wait, kErrTimeoutFull)) {
             ok = false;
