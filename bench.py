@@ -166,6 +166,18 @@ class ClockSampler:
 
 
 # ------------------------------------------------------------- timing ----
+def gpu_busy_before_start(dev, us=2000):
+    """Queue a short spin kernel (torch's, outside the timed region) so that
+    the GPU reaches the start event only after the host has queued the timed
+    work: a host-side hiccup (this process's clock-sampler thread, the GIL)
+    between recording the start event and launching the replay then adds no
+    idle GPU time to the measurement."""
+    sleep = getattr(torch.cuda, "_sleep", None)
+    if sleep is not None:
+        with torch.cuda.device(dev):
+            sleep(int(us * 2000))  # ~2 GHz SM clock: cycles for `us` microseconds
+
+
 class GraphTimer:
     """Captures ``n`` launches of a body over rotating operand sets into one
     CUDA graph and times ``replays`` replays separately with events on the
@@ -191,6 +203,7 @@ class GraphTimer:
         us = []
         for _ in range(replays):
             a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            gpu_busy_before_start(self.dev)
             a.record(self.stream)
             g.replay()
             b.record(self.stream)
@@ -324,6 +337,7 @@ def bench_device(args, rank, world, dev):
         w0 = time.perf_counter()
         t_start = torch.cuda.Event(enable_timing=True)
         t_end = torch.cuda.Event(enable_timing=True)
+        gpu_busy_before_start(dev)
         t_start.record(stream)
         for _ in range(full):
             graph.replay()
