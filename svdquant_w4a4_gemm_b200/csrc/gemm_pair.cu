@@ -20,12 +20,12 @@
 //   warps 0-1   producers: this CTA's 128 rows of A, its 96 rows of B (L2ᵀ on
 //               low-rank steps), the scales of its A rows and of all 192 B
 //               rows (each SM's tensor memory holds the B scales of the whole
-//               tile), with plain (non-multicast) TMA and bulk copies into
-//               its own shared memory, on its own barriers.
+//               tile), with plain TMA and bulk copies into its own shared
+//               memory, on its own barriers.
 //   warp 2      TMEM: both CTAs allocate the pair's 512 columns together; in
 //               rank 0, one thread issues the pair MMAs and commits them to the
-//               barriers of both CTAs at once (slot free, scale region free,
-//               accumulator full).
+//               barriers of both CTAs (slot free, scale region free,
+//               accumulator full), one commit per CTA.
 //   warps 3-6   stagers: scales into this SM's tensor memory and the low-rank
 //               A operand in place, then an arrival on rank 0's barrier
 //               (count 8: four warps of each CTA), so the MMA thread's one
@@ -57,7 +57,6 @@ constexpr int kThreads = 32 * (kProducers + 1 + kStagerWarps + kEpiWarps);
 constexpr uint32_t kA = kBM * kBKBytes;            // 16 KB
 constexpr uint32_t kSfa = 4 * 512;                 // this CTA's row block, 4 K-blocks
 constexpr uint32_t kBoxBytes = 32 * 128;           // 32 rows x 64 bf16
-constexpr uint16_t kPair = 0x3;                    // CTA mask of both CTAs
 
 // Sizes of a pair tile 256 x BN (BN = 128 or 192).
 template <int BN>
@@ -283,8 +282,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
               umma_nvfp4_pair(acc, da + 2 * kk, db + 2 * kk, id_fp4, sfr + 4 * kk,
                               sfr + 16 + kSfbCols * kk, (st > 0 || kk > 0) ? 1u : 0u);
           }
-          umma_commit_pair(&empty[s], kPair);
-          umma_commit_pair(&sffree[rg], kPair);
+          umma_commit_pair(&empty[s]);
+          umma_commit_pair(&sffree[rg]);
           rg = rg_next;
           sfr = rg == 0 ? tmem + kSfCol : sfr + kSfRegionCols;
           advance();
@@ -303,13 +302,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             umma_f16_pair(acc, da + 2 * kk, db + 2 * kk, id_f16, 1u);
             umma_f16_pair(acc, da + 2 * (2 + kk), db + 2 * kk, id_f16, 1u);
           }
-          umma_commit_pair(&empty[s], kPair);
+          umma_commit_pair(&empty[s]);
           advance();
         }
-        if (ok) umma_commit_pair(&acc_full[a], kPair);
+        if (ok) umma_commit_pair(&acc_full[a]);
       }
       // arrives once everything issued above has completed
-      umma_commit_pair(done, kPair);
+      umma_commit_pair(done);
     }
   } else if (warp < kMmaWarp + 1 + kStagerWarps) {
     // ----------------------------------------------------------- stagers ----

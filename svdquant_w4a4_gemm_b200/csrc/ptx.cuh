@@ -347,13 +347,19 @@ __device__ __forceinline__ void umma_nvfp4_pair(uint32_t d_tmem, uint64_t a_desc
       "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
       : "memory");
 }
-// Arrive on the mbarrier at this shared offset in every CTA of `cta_mask`
-// once all prior tcgen05 ops of this thread have completed.
-__device__ __forceinline__ void umma_commit_pair(uint64_t* bar, uint16_t cta_mask) {
+// Arrive on the mbarrier at this shared offset in both CTAs of the pair
+// once all prior tcgen05 ops of this thread have completed: one commit to
+// this CTA's barrier and one to the other CTA's (its address mapped into the
+// cluster window).
+__device__ __forceinline__ void umma_commit_pair(uint64_t* bar) {
   asm volatile(
-      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
-          smem_u32(bar)),
-      "h"(cta_mask)
+      "{\n\t.reg .b32 rb, rp, me;\n\t"
+      "mov.u32 me, %%cluster_ctarank;\n\t"
+      "xor.b32 rp, me, 1;\n\t"
+      "mapa.shared::cluster.u32 rb, %0, me;\n\t"
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [rb];\n\t"
+      "mapa.shared::cluster.u32 rb, %0, rp;\n\t"
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [rb];\n\t}" ::"r"(smem_u32(bar))
       : "memory");
 }
 
