@@ -267,14 +267,18 @@ __global__ void __launch_bounds__(kThreads, 2)
 // smoothing scales (1/a, K floats) into shared memory, then each strip with
 // one 3-D TMA copy (the strip's K/256 chunks of 128 bytes x 16 rows, chunk
 // major, 128-byte swizzle) and two bulk copies (its scales and zeros) into a
-// ring of shared-memory slots as deep as shared memory allows (~170 KB in
-// flight per SM, so the whole HBM stream starts at once).  In a slot, 128-byte
+// ring of shared-memory slots as deep as shared memory allows (7 slots, ~190
+// KB in flight per SM at K = 3072, so a CTA's whole share of the HBM stream
+// is requested at once).  The weight stream goes out only after the
+// consumers have issued their loads of x, which would otherwise wait behind
+// it in the memory system.  In a slot, 128-byte
 // line c·16 + r holds chunk c of row r with its 16-byte units XOR-ed by r mod
 // 8, so ldmatrix reads of the same unit of 8 rows hit 8 distinct bank groups.
 //
 // Twelve consumer warps split K: warp w always takes the same K/12 range, so
 // its activation fragments (x̂ = x·(1/a), bf16 hi and lo) are built once, in
-// registers, from one batch of loads of x.  Per 64-wide group a lane takes
+// registers, from one batch of loads of x (a warp with fewer than GMAX
+// groups runs the missing ones on zero fragments).  Per 64-wide group a lane takes
 // one ldmatrix.x4 (rows g and g+8, both 32-wide halves: 4 words of 8
 // nibbles), turns nibble pairs (i, i+4) into bf16 pairs 128 + q with one
 // LOP3 and into exact q − z with one bf16x2 subtract, and issues 4

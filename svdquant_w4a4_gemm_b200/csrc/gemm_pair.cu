@@ -96,7 +96,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   using L = PairLayout<BN>;
   constexpr int kBN = BN, kBHalf = L::kBHalf, kStages = L::kStages, kRegions = L::kRegions,
                 kBoxes = L::kBoxes;
-  constexpr uint32_t kB = L::kB, kSfb = L::kSfb, kStage = L::kStage, kRing = L::kRing, kBias = L::kBias,
+  constexpr uint32_t kB = L::kB, kStage = L::kStage, kRing = L::kRing, kBias = L::kBias,
                      kSfbCols = L::kSfbCols, kSfRegionCols = L::kSfRegionCols, kSfCol = L::kSfCol;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
