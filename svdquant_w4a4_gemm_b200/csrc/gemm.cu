@@ -48,6 +48,12 @@
 //               clipped at the M and N edges) into the tile's output (one,
 //               or one of up to three parts: Q, K, V of a fused
 //               projection); then release the accumulator.
+// Every CTA initialises its barriers, allocates tensor memory and prefetches
+// its descriptors before griddepcontrol.wait, so with programmatic dependent
+// launch that set-up overlaps the previous kernel's tail.  A step needs 46
+// KB of operands per SM from L2 at BN = 192, more than TMA delivers in the
+// 384 cycles of its four MMAs when every SM streams: the operand feed, not
+// the tensor pipe, sets the step time.
 #include "gemm_common.cuh"
 
 namespace svdq {

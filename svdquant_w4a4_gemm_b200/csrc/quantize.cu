@@ -15,9 +15,10 @@
 //                of L1ᵀ into a shared-memory ring as deep as shared memory
 //                allows, up to 8 sub-tiles (the loads come from HBM, and the
 //                ring must cover its latency).  The first loads of the ring
-//                are issued before the CTA-wide set-up, while
-//                the other warps compute RN(1/s) once for every column this
-//                CTA's range touches.
+//                go out as soon as the other warps have issued their own
+//                set-up loads (s and gs; behind the x stream they would
+//                wait microseconds), while those warps compute RN(1/s) once
+//                for every column this CTA's range touches.
 //   warp 1       TMEM owner; one thread issues the down-projection as
 //                tcgen05 kind::f16 MMAs (M = 128, N = r, K = 16 each) from
 //                the quantized tile's bf16(x̂) and the L1ᵀ slice into a TMEM
@@ -46,7 +47,10 @@
 //                a row block's K range can span several CTAs), then release
 //                the accumulator.
 // HBM traffic is the algorithmic minimum: x once, codes + scales + xl once;
-// L1ᵀ slices come from L2.
+// L1ᵀ slices come from L2.  xl is cleared by a small kernel launched just
+// before (clear_kernel, chained by programmatic dependent launch), and each
+// quantizer warp writes its 32 rows of codes through a shared-memory staging
+// area, so that a store covers whole 32-byte rows.
 //
 // Single-pass dynamic scale (gs_a = 2688 / max|x̂| computed in the same
 // launch): every CTA first streams its sub-tiles once for the max (phase A;
