@@ -169,3 +169,24 @@ def test_wait_timeout_setter_round_trips():
     prev = L.svdq_set_wait_timeout_ns(12345)
     assert L.svdq_set_wait_timeout_ns(0) == 12345
     L.svdq_set_wait_timeout_ns(prev)
+
+
+def test_launch_switches_round_trip_and_normalise():
+    """svdq_set_pdl and svdq_set_gemm_pairs are host-only: they return the
+    previous setting and store any non-zero value as 1 (defaults: PDL on,
+    pairs off)."""
+    L = sv.lib()
+    for setter, default in ((L.svdq_set_pdl, 1), (L.svdq_set_gemm_pairs, 0)):
+        prev = setter(7)
+        try:
+            assert prev == default
+            assert setter(0) == 1
+            assert setter(0) == 0
+        finally:
+            setter(prev)
+    # the Python wrappers report booleans
+    prev = sv.set_pdl(False)
+    try:
+        assert sv.set_pdl(True) is False
+    finally:
+        sv.set_pdl(prev)
