@@ -268,6 +268,11 @@ svdq_status svdq_w4a4_linear_split(const uint8_t* q_act, const uint8_t* sf_act,
  *   bias_bf16     [N] bf16 or NULL.
  *   N             N >= 16, N % 16 == 0.
  *   y_bf16        [M, N] bf16, contiguous.
+ *   Results do not depend on the kernel chosen beyond fp32 summation order:
+ *   K % 256 == 0, K <= 3072, scales and zeros 16-byte aligned and at most
+ *   16 row strips of 16 per SM go to a weight-streaming kernel (16-row
+ *   strips through a shared-memory ring by TMA); every other shape to a
+ *   register-streaming kernel, which sets the K limits above.
  *   Errors: INVALID_ARG, MISALIGNED, UNSUPPORTED_DEVICE, CUDA.
  */
 svdq_status awq_w4a16_linear(const void* x_bf16, int64_t M, int64_t K,
