@@ -738,17 +738,19 @@ def run_reference(args, rank, world, budget_s=90.0):
     actually timed and the ones requested)."""
     if rank != 0:
         return
+    from threadpoolctl import threadpool_limits
     rows = 32
     run = oracle_sample(rows)
-    t0 = time.perf_counter()
-    for _ in range(args.warmup):
-        run()
-    per = (time.perf_counter() - t0) / max(1, args.warmup)
-    steps = max(1, min(args.steps, int(budget_s / max(per, 1e-6))))
-    t0 = time.perf_counter()
-    for _ in range(steps):
-        run()
-    dt = (time.perf_counter() - t0) / steps
+    with threadpool_limits(limits=_CORES):
+        t0 = time.perf_counter()
+        for _ in range(args.warmup):
+            run()
+        per = (time.perf_counter() - t0) / max(1, args.warmup)
+        steps = max(1, min(args.steps, int(budget_s / max(per, 1e-6))))
+        t0 = time.perf_counter()
+        for _ in range(steps):
+            run()
+        dt = (time.perf_counter() - t0) / steps
     fl = layer_flops(rows, CASE.K, CASE.N, CASE.r)
     v = fl / dt / 1e12
     line = {"impl": "reference", "metric": METRIC, "value": v, "unit": UNIT, "n_gpus": world,
