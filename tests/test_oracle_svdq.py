@@ -28,6 +28,35 @@ def test_block_round_trip_of_representable_values():
     assert np.array_equal(svdq.nvfp4_dequantize(got_codes, got_sf, gs), x)
 
 
+def _worked_groups():
+    from tests._golden import rows
+    groups, cur = [], None
+    for r in rows("nvfp4_group_worked.txt"):
+        if r[0] == "case":
+            kv = dict(t.split("=", 1) for t in r[2:])
+            cur = dict(name=r[1], gs=np.float32(kv["gs"]), sf=int(kv["sf"], 16), x=[], codes=[])
+            groups.append(cur)
+        else:
+            cur["x"].append(np.float32(r[0]))
+            cur["codes"].append(int(r[1], 16))
+    return groups
+
+
+@pytest.mark.parametrize("g", _worked_groups(), ids=lambda g: g["name"])
+def test_quantize_matches_groups_worked_by_hand(g):
+    # groups off the representable grid (a block scale between E4M3 points,
+    # elements between E2M1 points, saturation of both, a scale rounding to
+    # zero), so that a misplaced tensor scale (t = a/(6·gs), inv = d/gs), a
+    # dropped rounding step or a lost sign changes the bytes
+    x = np.zeros((1, 16), np.float32)
+    n = len(g["x"])
+    x[0, :n] = g["x"]
+    codes, sf = svdq.nvfp4_quantize(x, g["gs"])
+    assert int(sf[0, 0]) == g["sf"]
+    assert codes[0, :n].tolist() == g["codes"]
+    assert np.all(codes[0, n:] == 0)
+
+
 def test_quantization_error_within_format_bound():
     rng = _rng(2)
     x = workloads.to_bf16(rng.standard_normal((64, 256)).astype(np.float32) * 3)
