@@ -47,6 +47,34 @@ def test_int4_quantization_error_bound_and_range():
     assert np.mean(np.abs(deq - w) <= 0.5 * step + 1e-12) > 0.95
 
 
+def _awq_worked_groups():
+    from tests._golden import rows
+    groups, cur = [], None
+    for r in rows("awq_group_worked.txt"):
+        if r[0] == "case":
+            kv = dict(t.split("=", 1) for t in r[2:])
+            cur = dict(name=r[1], sc=float(kv["sc"]), z=int(kv["z"]), w=[], q=[])
+            groups.append(cur)
+        else:
+            cur["w"].append(float(r[0]))
+            cur["q"].append(int(r[1]))
+    return groups
+
+
+@pytest.mark.parametrize("g", _awq_worked_groups(), ids=lambda g: g["name"])
+def test_int4_quantize_matches_groups_worked_by_hand(g):
+    # a scale exact in fp16 with ties in both directions, and one that fp16
+    # rounds (moving a value off a tie): pins the zero point's sign, the
+    # half-to-even rounding and that the divisions use the stored fp16 scale
+    w = np.zeros((1, 64))
+    n = len(g["w"])
+    w[0, :n] = g["w"]
+    q, sc, z = awq.int4_quantize(w)
+    assert float(sc[0, 0]) == g["sc"] and float(z[0, 0]) == g["z"]
+    assert q[0, :n].tolist() == g["q"]
+    assert np.all(q[0, n:] == g["z"])
+
+
 def test_constant_group_uses_unit_scale():
     w = np.full((1, 64), 3.0)
     q, sc, z = awq.int4_quantize(w)
