@@ -47,10 +47,10 @@ def test_int4_quantization_error_bound_and_range():
     assert np.mean(np.abs(deq - w) <= 0.5 * step + 1e-12) > 0.95
 
 
-def _awq_worked_groups():
+def _awq_groups_by_hand():
     from tests._golden import rows
     groups, cur = [], None
-    for r in rows("awq_group_worked.txt"):
+    for r in rows("awq_groups_by_hand.txt"):
         if r[0] == "case":
             kv = dict(t.split("=", 1) for t in r[2:])
             cur = dict(name=r[1], sc=float(kv["sc"]), z=int(kv["z"]), w=[], q=[])
@@ -61,8 +61,8 @@ def _awq_worked_groups():
     return groups
 
 
-@pytest.mark.parametrize("g", _awq_worked_groups(), ids=lambda g: g["name"])
-def test_int4_quantize_matches_groups_worked_by_hand(g):
+@pytest.mark.parametrize("g", _awq_groups_by_hand(), ids=lambda g: g["name"])
+def test_int4_quantize_matches_hand_quantized_groups(g):
     # a scale exact in fp16 with ties in both directions, and one that fp16
     # rounds (moving a value off a tie): pins the zero point's sign, the
     # half-to-even rounding and that the divisions use the stored fp16 scale

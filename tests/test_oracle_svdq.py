@@ -28,10 +28,10 @@ def test_block_round_trip_of_representable_values():
     assert np.array_equal(svdq.nvfp4_dequantize(got_codes, got_sf, gs), x)
 
 
-def _worked_groups():
+def _nvfp4_groups_by_hand():
     from tests._golden import rows
     groups, cur = [], None
-    for r in rows("nvfp4_group_worked.txt"):
+    for r in rows("nvfp4_groups_by_hand.txt"):
         if r[0] == "case":
             kv = dict(t.split("=", 1) for t in r[2:])
             cur = dict(name=r[1], gs=np.float32(kv["gs"]), sf=int(kv["sf"], 16), x=[], codes=[])
@@ -42,8 +42,8 @@ def _worked_groups():
     return groups
 
 
-@pytest.mark.parametrize("g", _worked_groups(), ids=lambda g: g["name"])
-def test_quantize_matches_groups_worked_by_hand(g):
+@pytest.mark.parametrize("g", _nvfp4_groups_by_hand(), ids=lambda g: g["name"])
+def test_quantize_matches_hand_quantized_groups(g):
     # groups off the representable grid (a block scale between E4M3 points,
     # elements between E2M1 points, saturation of both, a scale rounding to
     # zero), so that a misplaced tensor scale (t = a/(6·gs), inv = d/gs), a
