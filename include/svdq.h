@@ -79,12 +79,15 @@ size_t svdq_nvfp4_scale_bytes(int64_t rows, int64_t K);
  * that quantizes the activations; blog.margrop.com "技术细节 §1" step 4).
  *
  *   x_bf16      [M, K] bf16, row stride ldx elements (ldx >= K, ldx % 8 == 0).
- *   M, K        M >= 1, K >= 64, K % 64 == 0.
+ *   M, K        1 <= M <= 2^30; K >= 64, K % 64 == 0, and K within the
+ *               quantize kernel's shared memory (227 KB): K <= 47360 at
+ *               r = 0, 46336 at 16, 45312 at 32, 43264 at 64, 39168 at 128.
  *   smooth_s    [K] fp32 smoothing vector s (> 0), 4-byte aligned.  The
  *               kernel multiplies x by RN_fp32(1/s_k).  NULL = no smoothing.
  *   L1t_bf16    L1ᵀ, [r, K] bf16 row-major (K contiguous).  Ignored if r == 0.
  *   r           low-rank rank: 0 (no branch), 16, 32, 64 or 128.
- *   act_gscale  fp32 device scalar gs_a (static tensor scale).  NULL =
+ *   act_gscale  fp32 device scalar gs_a (static tensor scale), 4-byte
+ *               aligned (as is act_gscale_out).  NULL =
  *               dynamic: gs_a = 2688 / max|x̂| (1 if that max is 0), computed
  *               on the device by an extra pass over x.
  *   act_gscale_out  fp32 device scalar that receives the gs_a used; may alias
@@ -184,11 +187,12 @@ svdq_status svdq_quantize_act_dynamic_noalloc(const void* x_bf16, int64_t M, int
  *   lora_act    [M, r] fp32 (svdq_quantize_act's lora_out).  Ignored if r == 0.
  *   q_w         [N, K/2] E2M1 codes of the residual R (same packing).
  *   sf_w        svdq_nvfp4_scale_bytes(N, K) bytes, same layout.
- *   w_gscale    fp32 device scalar gs_w.
+ *   w_gscale    fp32 device scalar gs_w (4-byte aligned, as is act_gscale).
  *   L2t_bf16    L2ᵀ, [N, r] bf16 row-major (r contiguous).  Ignored if r == 0.
  *   r           0, 16, 32, 64 or 128.
- *   bias_bf16   [N] bf16 or NULL.
- *   M, N, K     M >= 1; N >= 16, N % 16 == 0; K >= 64, K % 64 == 0.
+ *   bias_bf16   [N] bf16 (2-byte aligned) or NULL.
+ *   M, N, K     1 <= M <= 2^30; 16 <= N <= 2^30, N % 16 == 0;
+ *               64 <= K <= 2^20, K % 64 == 0.
  *   y_bf16      [M, N] bf16, row stride ldy elements (ldy >= N, ldy % 8 == 0).
  *   Errors: INVALID_ARG, MISALIGNED, UNSUPPORTED_DEVICE, CUDA.
  */
@@ -263,11 +267,12 @@ svdq_status svdq_w4a4_linear_split(const uint8_t* q_act, const uint8_t* sf_act,
  *                 aligned, or NULL.
  *   qweight       [N, K/8] uint32, 16-byte aligned: nibble j (bits 4j..4j+3)
  *                 of word w of row n is q[n, 8w + j], an unsigned 0..15.
- *   scales_f16, zeros_f16   [N, K/group] fp16; zeros hold integers 0..15.
+ *   scales_f16, zeros_f16   [N, K/group] fp16, 2-byte aligned; zeros hold
+ *                 integers 0..15.
  *   group         must be 64.
- *   bias_bf16     [N] bf16 or NULL.
- *   N             N >= 16, N % 16 == 0.
- *   y_bf16        [M, N] bf16, contiguous.
+ *   bias_bf16     [N] bf16 (2-byte aligned) or NULL.
+ *   N             16 <= N <= 2^30, N % 16 == 0.
+ *   y_bf16        [M, N] bf16, contiguous, 2-byte aligned.
  *   Results do not depend on the kernel chosen beyond fp32 summation order:
  *   K % 256 == 0, K <= 3072, scales and zeros 16-byte aligned and at most
  *   16 row strips of 16 per SM go to a weight-streaming kernel (16-row

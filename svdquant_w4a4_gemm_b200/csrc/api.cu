@@ -279,9 +279,13 @@ svdq_status quantize_entry(const void* x_bf16, int64_t M, int64_t K, int64_t ldx
     return fail(SVDQ_ERR_INVALID_ARG, "r > 0 needs L1t_bf16 and lora_out");
   if (!act_gscale && !act_gscale_out)
     return fail(SVDQ_ERR_INVALID_ARG, "dynamic scale (act_gscale == NULL) needs act_gscale_out");
-  if (quantize_smem_bytes(K, r) > 227 * 1024 - 64)  // the opt-in limit less the static words
-    return fail(SVDQ_ERR_INVALID_ARG, "K=%lld with r=%d needs more than 227 KB of shared memory "
-                "(about K <= 24800 at r = 128, 37100 at r = 32)", (long long)K, r);
+  constexpr size_t kQuantSmemLimit = 227 * 1024 - 64;  // the opt-in limit less the static words
+  if (quantize_smem_bytes(K, r) > kQuantSmemLimit) {
+    int64_t kmax = K;  // the largest K this rank allows (error path only)
+    while (kmax > 64 && quantize_smem_bytes(kmax, r) > kQuantSmemLimit) kmax -= 64;
+    return fail(SVDQ_ERR_INVALID_ARG, "K=%lld with r=%d needs more than 227 KB of shared memory (K <= %lld at r=%d)",
+                (long long)K, r, (long long)kmax, r);
+  }
   if (!aligned16(x_bf16) || !aligned16(q_out) || !aligned16(sf_out) ||
       (r > 0 && (!aligned16(L1t_bf16) || !aligned16(lora_out))))
     return fail(SVDQ_ERR_MISALIGNED, "x, L1t, q_out, sf_out and lora_out must be 16-byte aligned");

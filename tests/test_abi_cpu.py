@@ -101,6 +101,40 @@ def test_smooth_s_needs_only_4_byte_alignment(monkeypatch):
     assert _q(s=18) == sv.MISALIGNED
 
 
+# The largest K the quantize call accepts at each rank (its kernel's shared
+# memory), as include/svdq.h states them.
+QUANT_KMAX = {0: 47360, 16: 46336, 32: 45312, 64: 43264, 128: 39168}
+
+
+@pytest.mark.parametrize("r", sorted(QUANT_KMAX))
+def test_quantize_k_limit_per_rank_is_the_headers(r, monkeypatch):
+    # a forced unsupported capability stops a valid call at the device check
+    monkeypatch.setenv("SVDQ_TEST_FORCE_CC", "9.0")
+    kmax = QUANT_KMAX[r]
+    lr = dict(L1t=16, lora=16) if r else {}
+    assert _q(K=kmax, ldx=kmax, r=r, **lr) == sv.UNSUPPORTED_DEVICE
+    assert _q(K=kmax + 64, ldx=kmax + 64, r=r, **lr) == sv.INVALID_ARG
+    assert f"K <= {kmax} at r={r}".encode() in sv.lib().svdq_last_error_detail()
+    with open(os.path.join(ROOT, "include", "svdq.h")) as f:
+        assert str(kmax) in f.read()
+
+
+def test_size_ceilings_are_validated(monkeypatch):
+    monkeypatch.setenv("SVDQ_TEST_FORCE_CC", "9.0")
+    assert _q(M=1 << 30) == sv.UNSUPPORTED_DEVICE
+    assert _q(M=(1 << 30) + 1) == sv.INVALID_ARG
+    L = sv.lib()
+    v = ctypes.c_void_p
+
+    def lin(M, N, K):
+        return L.svdq_w4a4_linear(v(16), v(16), v(16), None, v(16), v(16), v(16), None, 0, None,
+                                  M, N, K, v(16), N, None)
+    assert lin(4, 32, 1 << 20) == sv.UNSUPPORTED_DEVICE
+    assert lin(4, 32, (1 << 20) + 64) == sv.INVALID_ARG
+    assert lin((1 << 30) + 1, 32, 64) == sv.INVALID_ARG
+    assert lin(4, (1 << 30) + 16, 64) == sv.INVALID_ARG
+
+
 def test_single_pass_dynamic_quantize_validation_is_host_side():
     L = sv.lib()
     v = ctypes.c_void_p
