@@ -328,9 +328,11 @@ int svdq_set_gemm_pairs(int enable);
  * that kernel to complete and its writes to be visible (griddepcontrol.wait)
  * before it touches any operand in global memory, so every argument keeps
  * plain stream-order semantics.  Each kernel also signals at its start that
- * the next one may be scheduled.  0 launches in plain stream order.  The
- * pages have no counterpart (this is a launch property of the B200
- * implementation).  Returns the previous setting.  Host-only; never fails.
+ * the next one may be scheduled.  0 launches in plain stream order.
+ * awq_w4a16_linear with M > 4 always launches in plain stream order (it
+ * measured slower on B200 with the attribute).  The pages have no
+ * counterpart (this is a launch property of the B200 implementation).
+ * Returns the previous setting.  Host-only; never fails.
  */
 int svdq_set_pdl(int enable);
 

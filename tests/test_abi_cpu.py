@@ -202,7 +202,8 @@ def test_wait_timeout_setter_round_trips():
     L = sv.lib()
     prev = L.svdq_set_wait_timeout_ns(12345)
     assert L.svdq_set_wait_timeout_ns(0) == 12345
-    L.svdq_set_wait_timeout_ns(prev)
+    # 0 restores the documented default of 2 s
+    assert L.svdq_set_wait_timeout_ns(prev) == 2_000_000_000
 
 
 def test_launch_switches_round_trip_and_normalise():
