@@ -81,6 +81,13 @@ def _check(status):
         raise SvdqError(status, lib().svdq_last_error_detail().decode())
 
 
+def _require(cond, what):
+    # argument checks the C ABI cannot make (dtypes, strides); explicit, so
+    # that they hold under ``python -O`` too
+    if not cond:
+        raise ValueError(what)
+
+
 def _ptr(t):
     return None if t is None else ctypes.c_void_p(t.data_ptr())
 
@@ -123,7 +130,8 @@ def quantize_act(x, smooth=None, L1t=None, gscale=None, *, out=None):
     sf (scale bytes) uint8, lora [M, r] fp32 or None, gs fp32 [1]).
     ``out`` may pass preallocated (q, sf, lora, gs).
     """
-    assert x.dtype == torch.bfloat16 and x.dim() == 2 and x.stride(1) == 1
+    _require(x.dtype == torch.bfloat16 and x.dim() == 2 and x.stride(1) == 1,
+             "x must be a 2-D bf16 tensor with unit column stride")
     M, K = x.shape
     r = 0 if L1t is None else L1t.shape[0]
     dev = x.device
@@ -147,7 +155,8 @@ def quantize_act_dynamic(x, smooth=None, L1t=None, *, out=None, workspace=None):
     (one cooperative launch with a grid barrier).  ``workspace``: a device
     buffer of at least QUANTIZE_WORKSPACE_BYTES bytes, 16-byte aligned (one is
     allocated if None); calls that may overlap on the GPU need their own."""
-    assert x.dtype == torch.bfloat16 and x.dim() == 2 and x.stride(1) == 1
+    _require(x.dtype == torch.bfloat16 and x.dim() == 2 and x.stride(1) == 1,
+             "x must be a 2-D bf16 tensor with unit column stride")
     M, K = x.shape
     r = 0 if L1t is None else L1t.shape[0]
     dev = x.device
@@ -160,7 +169,8 @@ def quantize_act_dynamic(x, smooth=None, L1t=None, *, out=None, workspace=None):
         q, sf, lora, gs = out
     if workspace is None:
         workspace = torch.empty((QUANTIZE_WORKSPACE_BYTES,), dtype=torch.uint8, device=dev)
-    assert workspace.numel() * workspace.element_size() >= QUANTIZE_WORKSPACE_BYTES
+    _require(workspace.numel() * workspace.element_size() >= QUANTIZE_WORKSPACE_BYTES,
+             f"workspace must hold at least {QUANTIZE_WORKSPACE_BYTES} bytes")
     _check(lib().svdq_quantize_act_dynamic(_ptr(x), M, K, x.stride(0), _ptr(smooth), _ptr(L1t), r,
                                            _ptr(gs), _ptr(workspace), _ptr(q), _ptr(sf), _ptr(lora),
                                            _stream(dev)))
@@ -197,6 +207,7 @@ _ACTS = {None: ACT_NONE, "gelu": ACT_GELU_TANH}
 
 def w4a4_linear(q, sf, gs_a, lora, w: SvdqWeights, *, y=None, act=None):
     """y [M, N] bf16 = act(dec(q)·dec(W)ᵀ + lora·L2 + bias); act None or "gelu" (tanh form)."""
+    _require(act in _ACTS, f"act={act!r} must be None or 'gelu'")
     M, K = q.shape[0], q.shape[1] * 2
     N, r = w.N, w.rank
     if y is None:
@@ -211,6 +222,7 @@ def w4a4_linear(q, sf, gs_a, lora, w: SvdqWeights, *, y=None, act=None):
 def w4a4_linear_split(q, sf, gs_a, lora, w: SvdqWeights, parts=3, *, ys=None, act=None):
     """The fused projection stored as ``parts`` outputs [M, N/parts] bf16 (Q, K, V of a
     fused QKV projection): columns [i·N/parts, (i+1)·N/parts) of y go to ys[i]."""
+    _require(act in _ACTS, f"act={act!r} must be None or 'gelu'")
     M, K = q.shape[0], q.shape[1] * 2
     N, r = w.N, w.rank
     n_part = N // parts
@@ -218,7 +230,8 @@ def w4a4_linear_split(q, sf, gs_a, lora, w: SvdqWeights, parts=3, *, ys=None, ac
         ys = [torch.empty((M, n_part), dtype=torch.bfloat16, device=q.device) for _ in range(parts)]
     ys = list(ys)
     ldy = ys[0].stride(0)
-    assert len(ys) == parts and all(t.stride(0) == ldy and t.stride(1) == 1 for t in ys)
+    _require(len(ys) == parts and all(t.stride(0) == ldy and t.stride(1) == 1 for t in ys),
+             "ys must be `parts` row-major tensors with one leading dimension")
     arr = (_vp * parts)(*[_ptr(t) for t in ys])
     _check(lib().svdq_w4a4_linear_split(_ptr(q), _ptr(sf), _ptr(gs_a), _ptr(lora) if r else None,
                                         _ptr(w.q_w), _ptr(w.sf_w), _ptr(w.gs_w),
@@ -235,7 +248,7 @@ def svdq_linear(x, w: SvdqWeights, gscale=None, act=None):
 
 def awq_w4a16_linear(x, act_scale_inv, qweight, scales, zeros, bias=None, *, y=None, group=64):
     """y [M, N] bf16 for x [M <= 8, K] bf16 and int4 weights [N, K/8] uint32 (as int32)."""
-    assert x.dtype == torch.bfloat16 and x.is_contiguous()
+    _require(x.dtype == torch.bfloat16 and x.is_contiguous(), "x must be a contiguous bf16 tensor")
     M, K = x.shape
     N = qweight.shape[0]
     if y is None:
