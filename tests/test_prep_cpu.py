@@ -61,3 +61,30 @@ def test_the_prep_is_repeatable():
     b = randomized_svd(A, 16)
     for x, y in zip(a, b):
         assert torch.equal(x, y)
+
+
+def test_awq_prep_packs_and_quantizes_as_the_header_states():
+    # nibble j of word w holds q[n, 8w + j] (an int32 view of the uint32
+    # word, so words with the top nibble >= 8 are negative), zero points are
+    # integers, and (q - z)·sc is within half a step of W·diag(a) (no code of
+    # this draw meets the clamp to [0, 15], which could cost a step); the codes
+    # are the oracle's int4 quantizer's on the same scaled weights, except
+    # where fp32 and fp64 land on opposite sides of a rounding midpoint
+    from oracle import awq as oawq
+    from svdquant_w4a4_gemm_b200.prep import prepare_awq
+    rng = np.random.default_rng(11)
+    N, K = 48, 256
+    W = torch.from_numpy((rng.standard_normal((N, K)) * 0.05).astype(np.float32)).to(torch.bfloat16)
+    x_cal = torch.from_numpy(rng.standard_normal((64, K)).astype(np.float32)).to(torch.bfloat16)
+    ainv, words, sc, z = prepare_awq(W, x_cal)
+    assert words.dtype == torch.int32 and words.shape == (N, K // 8) and bool((words < 0).any())
+    q = oawq.unpack_int4_words(words.numpy().view(np.uint32), K).astype(np.float64)
+    zf, scf = z.double().numpy(), sc.double().numpy()
+    assert np.all(zf == np.rint(zf)) and zf.min() >= 0 and zf.max() <= 15
+    a = 1.0 / ainv.double().numpy()
+    target = W.double().numpy() * a[None, :]
+    deq = oawq.int4_dequantize(q.astype(np.uint8), sc.numpy(), z.numpy())
+    step = np.repeat(scf, 64, axis=1)
+    assert np.all(np.abs(deq - target) <= 0.5 * step * 1.01 + 1e-7)
+    q_ref, _, _ = oawq.int4_quantize(W.float().numpy().astype(np.float64) * (1.0 / ainv.numpy()).astype(np.float64))
+    assert np.mean(q_ref == q) > 0.999
