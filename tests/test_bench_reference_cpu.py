@@ -57,3 +57,14 @@ def test_reference_arm_other_ranks_exit_without_work():
     p = _run({"RANK": "1", "WORLD_SIZE": "2", "LOCAL_RANK": "1"}, "--steps", "1", "--warmup", "3")
     assert p.returncode == 0, p.stderr[-2000:]
     assert p.stdout.strip() == ""
+
+
+def test_roofline_numerators_are_the_algorithmic_counts():
+    # the headline layer M=4096, K=N=3072, r=32, counted by hand:
+    # FP4 GEMM 2·M·N·K = 77 309 411 328 and low-rank 2·M·r·(K+N) = 1 610 612 736
+    assert bench.layer_flops(4096, 3072, 3072, 32) == 78_920_024_064
+    # quantize: read x 25 165 824 + s 12 288 + L1ᵀ 196 608; write codes
+    # 6 291 456 + scales 786 432 + xl 524 288
+    assert bench.quantize_bytes(4096, 3072, 32) == 32_976_896
+    # no low-rank branch: no L1ᵀ and no xl
+    assert bench.quantize_bytes(4096, 3072, 0) == 32_976_896 - 196_608 - 524_288
