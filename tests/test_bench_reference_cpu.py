@@ -3,7 +3,9 @@ the host cores) keeps the bench line's contract: rank 0 prints exactly one
 JSON line carrying the same metric, unit, direction and workload as the
 library's own line, ``impl`` = "reference", a ``cpu_baseline`` object that
 describes the run and an ``e2e`` object with no host copies; every other
-rank exits 0 without work or output.  Runs on the CPU (no GPU needed)."""
+rank exits 0 without work or output.  Also: the roofline's numerators (the
+algorithmic FLOPs and bytes) are the hand-counted ones.  Runs on the CPU
+(no GPU needed)."""
 import json
 import os
 import subprocess
