@@ -44,7 +44,7 @@ def _gemm_on_oracle_inputs(case, smooth=True, with_bias=True, act=None, bias=Non
     return y, out["y"]
 
 
-# (M, K, N, r): BN=256 and BN=128 tiles, ragged M, ragged N tile, K not a
+# (M, K, N, r): BN=192 (N = 384) and BN=128 tiles, ragged M, ragged N tile, K not a
 # multiple of 256 (short last stage), every rank
 SMALL = [
     (128, 256, 256, 0),
