@@ -97,8 +97,8 @@ def test_quantize_mlp_down_full_size_sampled():
 
 
 # the ring depth follows K and r (as many 16 KB sub-tiles as shared memory
-# holds, at most 8): 8 at K=3072 for r <= 64, 6 at r=128; 7 and 5 at
-# K=12288 for r = 64 and 128.  Repeated runs must give the same bytes every
+# holds, rounded down to an even count, at most 8): 8 at K=3072 for r <= 64,
+# 6 at r=128; 6 and 4 at K=12288 for r = 64 and 128.  Repeated runs must give the same bytes every
 # time: a sub-tile quantized from a slot that does not yet hold it changes
 # the codes of that run only.
 @pytest.mark.parametrize("M,K,r", [(4608, 3072, 128), (4608, 3072, 32), (4096, 12288, 64),
